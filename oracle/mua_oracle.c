@@ -1,0 +1,300 @@
+/*
+ * MicroAdam step: plain single-threaded CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing in the product path may link, load or call
+ * this file: only the tests, the package's smoke check and the CPU-baseline leg
+ * of the benchmark do. It shares no code, header, table or constant generator
+ * with the CUDA path.
+ *
+ * Citations: [MicroAdam ¶n] is paragraph n of the web page "MicroAdam
+ * (Sparse-Gradient Adaptive Optimization with Quantized Error Feedback)":
+ *   ¶1 the per-step algorithm, ¶2 the state-memory formula, ¶3 Lemma 1 /
+ *   Lemma 3, ¶5 the update sparsity.
+ * Philox4x32-10 follows Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
+ * As Easy as 1, 2, 3" (SC'11).
+ *
+ * Precision. The quantities that decide an integer result (a_t, the Top-k
+ * order, delta/Delta and the 4-bit codes) are computed in fp32 with every
+ * operation rounded to nearest and no contraction (build with
+ * -ffp-contract=off), which is the precision the kernels decide them in.
+ * The window statistics m_hat, v_hat and the update are computed in fp64;
+ * parameters are stored in fp32 because that is their storage type.
+ *
+ * Readings of points the page leaves open (each also listed in the design
+ * notes):
+ *  - Q is uniform 4-bit stochastic rounding between the 16 levels
+ *    delta + c*(Delta-delta)/15, c = 0..15 (Lemma 1's (Delta-delta)/(2^b-1)
+ *    level spacing), with c = min(15, floor(s + xi)), s = (x - delta) *
+ *    (15/(Delta - delta)) and xi a 16-bit uniform draw in [0, 1).
+ *  - Top-k ties break to the lower index; a row lists its entries in
+ *    ascending index order; V is the signed value rounded to bf16 (RNE).
+ *  - m_hat = (1-beta1)/(1-beta1^t) * sum_r beta1^r V_r and likewise v_hat
+ *    with beta2 and V^2 (Adam's bias-corrected moments), r = age of the row.
+ *  - update u = m_hat / (eps + sqrt(v_hat)); decoupled weight decay
+ *    p <- p*(1 - lr*wd) is applied to every coordinate before the update.
+ *  - delta, Delta are global over the flat d-vector; blocks are cut over
+ *    that vector; a ragged last block of length L keeps
+ *    k = ceil(L*k_b/B_d) entries.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------------- */
+/* Philox4x32-10 (Salmon et al., SC'11): 10 rounds of the 4x32 S-box with  */
+/* multipliers M0, M1 and Weyl key increments W0, W1 between rounds.       */
+/* ---------------------------------------------------------------------- */
+#define PHILOX_M0 0xD2511F53u
+#define PHILOX_M1 0xCD9E8D57u
+#define PHILOX_W0 0x9E3779B9u
+#define PHILOX_W1 0xBB67AE85u
+
+void mua_oracle_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2],
+                              uint32_t out[4]) {
+    uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
+    uint32_t k0 = key_in[0], k1 = key_in[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += PHILOX_W0;
+            k1 += PHILOX_W1;
+        }
+        uint64_t prod0 = (uint64_t)PHILOX_M0 * (uint64_t)c0;
+        uint64_t prod1 = (uint64_t)PHILOX_M1 * (uint64_t)c2;
+        uint32_t hi0 = (uint32_t)(prod0 >> 32), lo0 = (uint32_t)prod0;
+        uint32_t hi1 = (uint32_t)(prod1 >> 32), lo1 = (uint32_t)prod1;
+        uint32_t n0 = hi1 ^ c1 ^ k0;
+        uint32_t n1 = lo1;
+        uint32_t n2 = hi0 ^ c3 ^ k1;
+        uint32_t n3 = lo0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* The 16-bit uniform draw used for element i at step t: Philox with key =
+ * seed and counter = (i/8 low, i/8 high, t low, t high); element i takes the
+ * (i mod 2)-th 16-bit half of output word (i/2) mod 4. */
+uint32_t mua_oracle_draw16(uint64_t seed, int64_t t, int64_t i) {
+    uint64_t j = (uint64_t)i >> 3;
+    uint32_t ctr[4] = {(uint32_t)j, (uint32_t)(j >> 32), (uint32_t)(uint64_t)t,
+                       (uint32_t)((uint64_t)t >> 32)};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    mua_oracle_philox4x32_10(ctr, key, out);
+    uint32_t word = out[((uint64_t)i >> 1) & 3];
+    return (i & 1) ? (word >> 16) : (word & 0xFFFFu);
+}
+
+/* ---------------------------------------------------------------------- */
+/* bfloat16: the top 16 bits of an IEEE binary32.                          */
+/* ---------------------------------------------------------------------- */
+static float f32_from_bits(uint32_t b) { float f; memcpy(&f, &b, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t b; memcpy(&b, &f, 4); return b; }
+
+float mua_oracle_bf16_to_f32(uint16_t h) { return f32_from_bits((uint32_t)h << 16); }
+
+/* Round to nearest, ties to even, on the 16 discarded bits; NaN stays NaN. */
+uint16_t mua_oracle_f32_to_bf16(float f) {
+    uint32_t b = bits_from_f32(f);
+    if ((b & 0x7F800000u) == 0x7F800000u && (b & 0x007FFFFFu) != 0)
+        return (uint16_t)((b >> 16) | 0x0040u);
+    uint32_t lsb = (b >> 16) & 1u;
+    return (uint16_t)((b + 0x7FFFu + lsb) >> 16);
+}
+
+/* ---------------------------------------------------------------------- */
+/* The 4-bit codec Q / Q^{-1} [MicroAdam ¶1, ¶3 Lemma 1].                   */
+/* Codes are packed two per byte, element 2q in the low nibble of byte q.   */
+/* ---------------------------------------------------------------------- */
+static unsigned get_code(const uint8_t* codes, int64_t i) {
+    uint8_t byte = codes[i >> 1];
+    return (i & 1) ? (unsigned)(byte >> 4) : (unsigned)(byte & 0xFu);
+}
+
+static void put_code(uint8_t* codes, int64_t i, unsigned c) {
+    uint8_t byte = codes[i >> 1];
+    if (i & 1) byte = (uint8_t)((byte & 0x0Fu) | (c << 4));
+    else       byte = (uint8_t)((byte & 0xF0u) | c);
+    codes[i >> 1] = byte;
+}
+
+/* Q^{-1}(e, delta, Delta)_i = delta + c_i * (Delta - delta)/15, in fp32. */
+void mua_oracle_dequantize(const uint8_t* codes, int64_t n, float delta, float Delta,
+                           float* out) {
+    float unit = (Delta - delta) / 15.0f;
+    for (int64_t i = 0; i < n; ++i) {
+        float level = (float)get_code(codes, i) * unit;
+        out[i] = delta + level;
+    }
+}
+
+/* e = Q(x, delta, Delta): stochastic rounding of x onto the 16 levels.
+ * base is the global index of x[0] (it selects the random draws). */
+void mua_oracle_quantize(const float* x, int64_t n, int64_t base, float delta, float Delta,
+                         int64_t t, uint64_t seed, uint8_t* codes) {
+    float inv = (Delta == delta) ? 0.0f : 15.0f / (Delta - delta);
+    for (int64_t i = 0; i < n; ++i) {
+        float s = (x[i] - delta) * inv;
+        float xi = (float)mua_oracle_draw16(seed, t, base + i) * (1.0f / 65536.0f);
+        float y = s + xi;
+        unsigned c = 0;
+        if (y >= 1.0f) {
+            float f = floorf(y);
+            c = (f >= 15.0f) ? 15u : (unsigned)f;
+        }
+        put_code(codes, i, c);
+    }
+}
+
+/* ---------------------------------------------------------------------- */
+/* Per-block Top-k of |a| [MicroAdam ¶1].                                   */
+/* ---------------------------------------------------------------------- */
+typedef struct { uint32_t key; int32_t idx; } keyed_t;
+
+/* Order: larger |a| first; among equal |a|, the lower index first. */
+static int by_key_desc_idx_asc(const void* pa, const void* pb) {
+    const keyed_t* a = (const keyed_t*)pa;
+    const keyed_t* b = (const keyed_t*)pb;
+    if (a->key != b->key) return (a->key > b->key) ? -1 : 1;
+    return (a->idx < b->idx) ? -1 : (a->idx > b->idx);
+}
+
+static int by_idx_asc(const void* pa, const void* pb) {
+    const keyed_t* a = (const keyed_t*)pa;
+    const keyed_t* b = (const keyed_t*)pb;
+    return (a->idx < b->idx) ? -1 : (a->idx > b->idx);
+}
+
+/* k for a block of length L: ceil(L * k_b / B_d). */
+int64_t mua_oracle_block_k(int64_t L, int32_t Bd, int32_t kb) {
+    return (L * (int64_t)kb + Bd - 1) / Bd;
+}
+
+/* ---------------------------------------------------------------------- */
+/* One MicroAdam step [MicroAdam ¶1], stages in the page's order.           */
+/*                                                                          */
+/* p      [d]            fp32 parameters, updated in place                  */
+/* g      [d]            bf16 gradient (raw bits)                           */
+/* codes  [ceil(d/2)]    e_t in, e_{t+1} out                                */
+/* scal   [2]            (delta_t, Delta_t) in, (delta_{t+1}, Delta_{t+1})  */
+/* G_idx  [m][n_b][k_b]  int16 block-relative indices, -1 = empty slot      */
+/* G_val  [m][n_b][k_b]  bf16 values (raw bits)                             */
+/* mhat, vhat, mabs [d]  optional (NULL = skip): m_hat, v_hat and the       */
+/*                       cancellation-free magnitude (1-b1)/(1-b1^t) *      */
+/*                       sum_r b1^r |V_r|; zero where no window entry.      */
+/* Returns 0, or -1 on bad arguments / allocation failure.                  */
+/* ---------------------------------------------------------------------- */
+int mua_oracle_step(int64_t d, int32_t Bd, int32_t kb, int32_t m, float* p,
+                    const uint16_t* g, uint8_t* codes, float* scal, int16_t* G_idx,
+                    uint16_t* G_val, double lr, double beta1, double beta2, double eps,
+                    double wd, int64_t t, uint64_t seed, double* mhat, double* vhat,
+                    double* mabs) {
+    if (d < 1 || Bd < 1 || Bd > 32766 || kb < 1 || kb > Bd || m < 1 || t < 1) return -1;
+    const int64_t nb = (d + Bd - 1) / Bd;
+    const float delta_t = scal[0], Delta_t = scal[1];
+
+    float* a = (float*)malloc(sizeof(float) * (size_t)d);
+    keyed_t* order = (keyed_t*)malloc(sizeof(keyed_t) * (size_t)Bd);
+    double* z1 = (double*)calloc((size_t)d, sizeof(double));
+    double* z2 = (double*)calloc((size_t)d, sizeof(double));
+    double* za = (double*)calloc((size_t)d, sizeof(double));
+    uint8_t* touched = (uint8_t*)calloc((size_t)d, 1);
+    if (!a || !order || !z1 || !z2 || !za || !touched) {
+        free(a); free(order); free(z1); free(z2); free(za); free(touched);
+        return -1;
+    }
+
+    /* (1) a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t). */
+    {
+        float unit = (Delta_t - delta_t) / 15.0f;
+        for (int64_t i = 0; i < d; ++i) {
+            float level = (float)get_code(codes, i) * unit;
+            float deq = delta_t + level;
+            a[i] = mua_oracle_bf16_to_f32(g[i]) + deq;
+        }
+    }
+
+    /* (2) (I_t, V_t) = T_k(|a_t|) per block, written to row t mod m of G;
+     * (3) the selected entries of a_t are set to zero. */
+    const int64_t row = t % m;
+    for (int64_t j = 0; j < nb; ++j) {
+        const int64_t start = j * (int64_t)Bd;
+        const int64_t L = (d - start < Bd) ? (d - start) : Bd;
+        const int64_t k = mua_oracle_block_k(L, Bd, kb);
+        for (int64_t q = 0; q < L; ++q) {
+            order[q].key = bits_from_f32(a[start + q]) & 0x7FFFFFFFu;
+            order[q].idx = (int32_t)q;
+        }
+        qsort(order, (size_t)L, sizeof(keyed_t), by_key_desc_idx_asc);
+        qsort(order, (size_t)k, sizeof(keyed_t), by_idx_asc);
+        int16_t* ri = G_idx + (row * nb + j) * kb;
+        uint16_t* rv = G_val + (row * nb + j) * kb;
+        for (int64_t s = 0; s < kb; ++s) {
+            if (s < k) {
+                int64_t q = order[s].idx;
+                ri[s] = (int16_t)q;
+                rv[s] = mua_oracle_f32_to_bf16(a[start + q]);
+            } else {
+                ri[s] = -1;
+                rv[s] = 0;
+            }
+        }
+        for (int64_t s = 0; s < k; ++s) a[start + order[s].idx] = 0.0f;
+    }
+
+    /* (4) e_{t+1} = Q(a_t, delta_{t+1}, Delta_{t+1}) with the scalar min and
+     * max of the residual (a -0 result is stored as +0). */
+    float lo = a[0], hi = a[0];
+    for (int64_t i = 1; i < d; ++i) {
+        if (a[i] < lo) lo = a[i];
+        if (a[i] > hi) hi = a[i];
+    }
+    lo = lo + 0.0f;
+    hi = hi + 0.0f;
+    mua_oracle_quantize(a, d, 0, lo, hi, t, seed, codes);
+    scal[0] = lo;
+    scal[1] = hi;
+
+    /* (5) m_hat = AdamStats(beta1, G), v_hat = AdamStats(beta2, G^2) by the
+     * unrolled decay z[I] += beta^r V over the rows in the window, oldest
+     * (largest age r) first. */
+    const int64_t rows = (t < m) ? t : m;
+    for (int64_t r = rows - 1; r >= 0; --r) {
+        const int64_t rr = (t - r) % m;
+        const double w1 = pow(beta1, (double)r);
+        const double w2 = pow(beta2, (double)r);
+        for (int64_t j = 0; j < nb; ++j) {
+            const int16_t* ri = G_idx + (rr * nb + j) * kb;
+            const uint16_t* rv = G_val + (rr * nb + j) * kb;
+            for (int64_t s = 0; s < kb; ++s) {
+                if (ri[s] < 0) continue;
+                const int64_t q = j * (int64_t)Bd + ri[s];
+                const double V = (double)mua_oracle_bf16_to_f32(rv[s]);
+                z1[q] += w1 * V;
+                z2[q] += w2 * (V * V);
+                za[q] += w1 * fabs(V);
+                touched[q] = 1;
+            }
+        }
+    }
+    const double f1 = (1.0 - beta1) / (1.0 - pow(beta1, (double)t));
+    const double f2 = (1.0 - beta2) / (1.0 - pow(beta2, (double)t));
+
+    /* (6) p <- p*(1 - lr*wd) - lr * m_hat / (eps + sqrt(v_hat)). */
+    const double decay = 1.0 - lr * wd;
+    for (int64_t q = 0; q < d; ++q) {
+        const double m_hat = f1 * z1[q];
+        const double v_hat = f2 * z2[q];
+        if (mhat) mhat[q] = m_hat;
+        if (vhat) vhat[q] = v_hat;
+        if (mabs) mabs[q] = f1 * za[q];
+        double pq = (double)p[q];
+        if (wd != 0.0) pq = pq * decay;
+        if (touched[q]) pq = pq - lr * (m_hat / (eps + sqrt(v_hat)));
+        if (wd != 0.0 || touched[q]) p[q] = (float)pq;
+    }
+
+    free(a); free(order); free(z1); free(z2); free(za); free(touched);
+    return 0;
+}
