@@ -1,0 +1,269 @@
+// Host side of libmua.so: the C ABI declared in include/mua.h.
+//
+// [MicroAdam ¶n] is paragraph n of "MicroAdam (Sparse-Gradient Adaptive
+// Optimization with Quantized Error Feedback)".
+//
+// A handle holds geometry only. mua_step enqueues, on the caller's stream:
+//   1. an 8-byte memset of the (-delta_{t+1}, Delta_{t+1}) accumulator pair,
+//   2. the select kernel (one CTA per block),
+//   3. the apply kernel (one CTA per block, reverse block order so the tail of
+//      the select kernel's reads is still in L2).
+// Everything the kernels need per step (beta^r weights, bias corrections,
+// Philox round keys) is computed here in fp64 and rounded once to fp32 /
+// uint32 before launch.
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/mua.h"
+#include "mua_kernels.cuh"
+
+struct mua_ctx {
+  int64_t d;            // elements of this handle
+  int64_t d_total;      // elements of the whole vector
+  int64_t block_begin;  // first global block
+  int64_t nb;           // blocks of this handle
+  int32_t Bd, kb, kp, m;
+  int32_t last_len;
+  int32_t threads;
+  bool vec;             // 16-byte vector path usable (B_d % 8 == 0)
+  int64_t off_codes, off_window, bytes;
+  uint32_t apply_smem;
+};
+
+namespace {
+
+thread_local char g_cuda_err[256] = "no CUDA error";
+
+int cuda_fail(cudaError_t e, const char* where) {
+  std::snprintf(g_cuda_err, sizeof g_cuda_err, "%s: %s", where, cudaGetErrorString(e));
+  return MUA_ERR_CUDA;
+}
+
+int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+int pick_threads(int Bd) {
+  const int need = (Bd + mua::kElemsPerThread - 1) / mua::kElemsPerThread;
+  int t = 32;
+  while (t < need) t <<= 1;
+  return t;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
+         int64_t block_begin, int64_t block_count, mua_t* out) {
+  if (!out) return MUA_ERR_ARG;
+  *out = nullptr;
+  if (d_total < 1 || Bd < 2 || Bd > 32766 || (Bd & 1) || kb < 1 || kb > Bd || m < 1 ||
+      m > mua::kMaxWindow)
+    return MUA_ERR_ARG;
+  if (bits != 4) return MUA_ERR_UNSUPPORTED;
+  const int64_t nb_total = (d_total + Bd - 1) / Bd;
+  if (block_begin < 0 || block_count < 1 || block_begin + block_count > nb_total)
+    return MUA_ERR_ARG;
+  if (block_count > 0x7FFFFFFF) return MUA_ERR_UNSUPPORTED;
+  const int32_t kp = (int32_t)round_up(kb, 4);
+  if ((int64_t)m * kp > mua::kMaxWindowEntries) return MUA_ERR_UNSUPPORTED;
+
+  mua_ctx* h = new (std::nothrow) mua_ctx();
+  if (!h) return MUA_ERR_ARG;
+  h->d_total = d_total;
+  h->block_begin = block_begin;
+  h->nb = block_count;
+  const int64_t first = block_begin * Bd;
+  const int64_t last_end = std::min<int64_t>(d_total, (block_begin + block_count) * Bd);
+  h->d = last_end - first;
+  h->Bd = Bd;
+  h->kb = kb;
+  h->kp = kp;
+  h->m = m;
+  h->last_len = (int32_t)(h->d - (block_count - 1) * Bd);
+  h->threads = pick_threads(Bd);
+  h->vec = (Bd % 8) == 0;
+  h->off_codes = 256;
+  h->off_window = h->off_codes + round_up((h->d + 1) / 2, 256);
+  h->bytes = h->off_window + 4 * block_count * (int64_t)m * kp;
+  h->apply_smem = mua::apply_smem_bytes(h->threads, Bd, kp, m);
+  *out = h;
+  return MUA_OK;
+}
+
+bool finite_f(float x) { return std::isfinite(x); }
+
+int check_hyper(float lr, float beta1, float beta2, float eps, float wd, int64_t t) {
+  if (t < 1) return MUA_ERR_ARG;
+  if (!finite_f(lr) || !finite_f(wd) || !finite_f(eps) || eps < 0.0f) return MUA_ERR_ARG;
+  if (!(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f)) return MUA_ERR_ARG;
+  return MUA_OK;
+}
+
+mua::Geometry geometry(const mua_ctx* h) {
+  mua::Geometry g;
+  g.d = h->d;
+  g.base_index = h->block_begin * h->Bd;
+  g.Bd = h->Bd;
+  g.kb = h->kb;
+  g.kp = h->kp;
+  g.m = h->m;
+  g.nb = (int32_t)h->nb;
+  g.last_len = h->last_len;
+  return g;
+}
+
+// Header word of the (-delta, Delta) pair holding step s's scalars.
+int pair_word(int64_t s) { return (s & 1) ? mua::kHdrPair1 : mua::kHdrPair0; }
+
+}  // namespace
+
+extern "C" {
+
+int mua_create(int64_t d, int32_t block_size, int32_t k_per_block, int32_t window,
+               int32_t bits, mua_t* out) {
+  if (d < 1 || block_size < 2) {
+    if (out) *out = nullptr;
+    return MUA_ERR_ARG;
+  }
+  return make(d, block_size, k_per_block, window, bits, 0, (d + block_size - 1) / block_size,
+              out);
+}
+
+int mua_create_shard(int64_t d_total, int32_t block_size, int32_t k_per_block, int32_t window,
+                     int32_t bits, int64_t block_begin, int64_t block_count, mua_t* out) {
+  return make(d_total, block_size, k_per_block, window, bits, block_begin, block_count, out);
+}
+
+void mua_destroy(mua_t h) { delete h; }
+
+int64_t mua_state_bytes(mua_t h) { return h ? h->bytes : MUA_ERR_ARG; }
+
+int mua_state_layout(mua_t h, int64_t* out) {
+  if (!h || !out) return MUA_ERR_ARG;
+  out[MUA_LAYOUT_HEADER] = 0;
+  out[MUA_LAYOUT_CODES] = h->off_codes;
+  out[MUA_LAYOUT_WINDOW] = h->off_window;
+  out[MUA_LAYOUT_ROW_STRIDE] = h->kp;
+  out[MUA_LAYOUT_BLOCKS] = h->nb;
+  out[MUA_LAYOUT_BYTES] = h->bytes;
+  return MUA_OK;
+}
+
+int64_t mua_minmax_offset(mua_t h, int64_t t) {
+  if (!h || t < 1) return MUA_ERR_ARG;
+  return 4 * (int64_t)pair_word(t + 1);
+}
+
+int mua_select(mua_t h, const uint16_t* grads, void* state, int64_t t, void* stream) {
+  if (!h || !grads || !state || t < 1) return MUA_ERR_ARG;
+  if (!aligned16(grads) || !aligned16(state)) return MUA_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* st = static_cast<uint8_t*>(state);
+  mua::SelectArgs A;
+  A.g = geometry(h);
+  A.grads = grads;
+  A.codes = st + h->off_codes;
+  A.window = reinterpret_cast<uint32_t*>(st + h->off_window);
+  A.hdr = reinterpret_cast<uint32_t*>(st);
+  A.row = (int32_t)(t % h->m);
+  A.pair_cur = pair_word(t);
+  A.pair_next = pair_word(t + 1);
+  cudaError_t e = cudaMemsetAsync(A.hdr + A.pair_next, 0, 8, s);
+  if (e != cudaSuccess) return cuda_fail(e, "reset of the min/max pair");
+  e = mua::launch_select(A, h->threads, h->vec, s);
+  if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  return MUA_OK;
+}
+
+int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
+              float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+              float* mhat, float* vhat, void* stream) {
+  if (!h || !params || !grads || !state) return MUA_ERR_ARG;
+  int rc = check_hyper(lr, beta1, beta2, eps, wd, t);
+  if (rc != MUA_OK) return rc;
+  if (!aligned16(params) || !aligned16(grads) || !aligned16(state)) return MUA_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* st = static_cast<uint8_t*>(state);
+  mua::ApplyArgs A;
+  std::memset(&A, 0, sizeof A);
+  A.g = geometry(h);
+  A.params = params;
+  A.grads = grads;
+  A.codes = st + h->off_codes;
+  A.window = reinterpret_cast<const uint32_t*>(st + h->off_window);
+  A.hdr = reinterpret_cast<uint32_t*>(st);
+  A.mhat = mhat;
+  A.vhat = vhat;
+  A.row = (int32_t)(t % h->m);
+  A.rows = (int32_t)std::min<int64_t>(t, h->m);
+  A.pair_cur = pair_word(t);
+  A.pair_next = pair_word(t + 1);
+  A.t_lo = (uint32_t)(uint64_t)t;
+  A.t_hi = (uint32_t)((uint64_t)t >> 32);
+  const double b1 = beta1, b2 = beta2;
+  A.lr = lr;
+  A.eps = eps;
+  A.decay = (float)(1.0 - (double)lr * (double)wd);
+  A.has_decay = (wd != 0.0f);
+  // Adam's bias correction of the unrolled sums [MicroAdam ¶1]:
+  // m_hat = (1-beta1)/(1-beta1^t) * sum_r beta1^r V_r, likewise v_hat.
+  A.f1 = (float)((1.0 - b1) / (1.0 - std::pow(b1, (double)t)));
+  A.f2 = (float)((1.0 - b2) / (1.0 - std::pow(b2, (double)t)));
+  for (int r = 0; r < mua::kMaxWindow; ++r) {
+    A.w1[r] = (float)std::pow(b1, (double)r);
+    A.w2[r] = (float)std::pow(b2, (double)r);
+  }
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    A.keys[r][0] = k0;
+    A.keys[r][1] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  A.reverse = 1;
+  A.smem_bytes = h->apply_smem;
+  const cudaError_t e = mua::launch_apply(A, h->threads, h->vec, s);
+  if (e != cudaSuccess) return cuda_fail(e, "apply kernel launch");
+  return MUA_OK;
+}
+
+int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float lr, float beta1,
+             float beta2, float eps, float wd, int64_t t, uint64_t seed, void* stream) {
+  if (!h || !params || !grads || !state) return MUA_ERR_ARG;
+  int rc = check_hyper(lr, beta1, beta2, eps, wd, t);
+  if (rc != MUA_OK) return rc;
+  if (!aligned16(params) || !aligned16(grads) || !aligned16(state)) return MUA_ERR_ALIGN;
+  rc = mua_select(h, grads, state, t, stream);
+  if (rc != MUA_OK) return rc;
+  return mua_apply(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, nullptr, nullptr,
+                   stream);
+}
+
+int mua_get_status(mua_t h, const void* state, uint32_t* out, void* stream) {
+  if (!h || !state || !out) return MUA_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint32_t* hdr = static_cast<const uint32_t*>(state);
+  cudaError_t e = cudaMemcpyAsync(out, hdr + mua::kHdrStatus, 4, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "status copy");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "status synchronize");
+  return MUA_OK;
+}
+
+const char* mua_strerror(int code) {
+  switch (code) {
+    case MUA_OK: return "ok";
+    case MUA_ERR_ARG: return "argument out of range or NULL";
+    case MUA_ERR_UNSUPPORTED: return "unsupported configuration (bits != 4 or window too large)";
+    case MUA_ERR_ALIGN: return "device pointer not 16-byte aligned";
+    case MUA_ERR_CUDA: return "CUDA runtime error (see mua_last_cuda_error)";
+    default: return "unknown error code";
+  }
+}
+
+const char* mua_last_cuda_error(void) { return g_cuda_err; }
+
+const char* mua_version(void) { return "mua 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -148,17 +148,33 @@ def _fill_grad(dst: torch.Tensor, kind: str, scale: float, g: torch.Generator):
 
 
 def make_grads(w: Workload, step: int, device="cpu", out: torch.Tensor | None = None,
-               chunk: int = 1 << 25) -> torch.Tensor:
-    """bf16 gradients of workload ``w`` for optimizer step ``step`` (seeded by both)."""
+               start: int = 0, length: int | None = None, chunk: int = 1 << 24) -> torch.Tensor:
+    """bf16 gradients of workload ``w`` for optimizer step ``step``.
+
+    Element i of tensor j draws from a generator seeded by (workload, step, j,
+    i // chunk), so any slice [start, start + length) of the flat vector is
+    reproducible on its own (one rank's shard) and equals the same slice of
+    the whole vector.
+    """
+    if length is None:
+        length = w.d - start
     if out is None:
-        out = torch.empty(w.d, dtype=torch.bfloat16, device=device)
-    g = _gen(out.device, 1000003 * (w.seed & 0xFFFF) + 7919 * step + 17)
+        out = torch.empty(length, dtype=torch.bfloat16, device=device)
+    assert out.numel() == length
+    end = start + length
     offset = 0
     for j, n in enumerate(w.tensor_sizes()):
-        scale = tensor_scale(j) if w.grad == "t3_tensor_scaled" else 1e-3
-        for s in range(0, n, chunk):
-            e = min(n, s + chunk)
-            _fill_grad(out[offset + s: offset + e], w.grad, scale, g)
+        lo, hi = max(start, offset), min(end, offset + n)
+        if lo < hi:
+            scale = tensor_scale(j) if w.grad == "t3_tensor_scaled" else 1e-3
+            for c in range((lo - offset) // chunk, (hi - offset - 1) // chunk + 1):
+                c0 = offset + c * chunk
+                c1 = min(offset + n, c0 + chunk)
+                g = _gen(out.device, ((w.seed * 1000003 + step) * 7919 + j) * 104729 + c)
+                buf = torch.empty(c1 - c0, dtype=torch.bfloat16, device=out.device)
+                _fill_grad(buf, w.grad, scale, g)
+                a, b = max(lo, c0), min(hi, c1)
+                out[a - start: b - start].copy_(buf[a - c0: b - c0])
         offset += n
     return out
 

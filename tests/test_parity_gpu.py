@@ -1,0 +1,187 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle, step by
+step, on the same seeded inputs.
+
+Bit-exact: the window rows (int16 I, bf16 V), the 4-bit codes, delta/Delta
+and the status word. Within 1e-5: the parameters (relative, with an absolute
+floor of 1e-5 * lr, the scale of one update), v_hat (relative) and m_hat
+(relative to the cancellation-free magnitude (1-b1)/(1-b1^t) sum b1^r |V|,
+since m_hat sums terms of both signs).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import state_view
+from conftest import cuda_available
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not cuda_available(), reason="needs a CUDA device")]
+
+RTOL = 1e-5
+
+
+def _mods():
+    import torch
+    from compressed_state_optimizer_b200 import MicroAdam, workloads
+    return torch, MicroAdam, workloads
+
+
+def compare_state(mo, state, ost, t, d, m, kb, what=""):
+    sb = state.cpu().numpy()
+    lay = mo.layout
+    assert np.array_equal(state_view.codes(sb, lay, d), ost.codes), f"codes differ {what} t={t}"
+    lo, hi = state_view.header_scalars(sb, t + 1)
+    assert np.float32(lo).view(np.uint32) == ost.scal[0:1].view(np.uint32)[0], (what, t, lo, ost.scal)
+    assert np.float32(hi).view(np.uint32) == ost.scal[1:2].view(np.uint32)[0], (what, t, hi, ost.scal)
+    gi, gv = state_view.window(sb, lay, m, kb)
+    for s in range(max(1, t - m + 1), t + 1):
+        r = s % m
+        assert np.array_equal(gi[r], ost.G_idx[r]), f"window indices differ {what} t={t} row step {s}"
+        assert np.array_equal(gv[r], ost.G_val[r]), f"window values differ {what} t={t} row step {s}"
+    return sb
+
+
+def compare_params(p_gpu, p_ref, lr, what=""):
+    p = p_gpu.cpu().numpy()
+    err = np.abs(p.astype(np.float64) - p_ref.astype(np.float64))
+    tol = RTOL * np.maximum(np.abs(p_ref.astype(np.float64)), lr)
+    bad = np.flatnonzero(err > tol)
+    assert bad.size == 0, f"params differ {what} at {bad[:5]}: {p[bad[:5]]} vs {p_ref[bad[:5]]}"
+
+
+def compare_stats(mhat, vhat, stats, what=""):
+    mh_ref, vh_ref, mabs = stats
+    mh = mhat.cpu().numpy().astype(np.float64)
+    vh = vhat.cpu().numpy().astype(np.float64)
+    touched = mabs > 0
+    assert np.all(mh[~touched] == 0) and np.all(vh[~touched] == 0), what
+    assert np.all(np.abs(mh - mh_ref) <= RTOL * mabs + 1e-30), what
+    assert np.all(np.abs(vh - vh_ref) <= RTOL * vh_ref + 1e-30), what
+
+
+def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0.9,
+               b2=0.999, eps=1e-8, wd=0.0, grads_fn=None, stats=True, use_step=False):
+    torch, MicroAdam, workloads = _mods()
+    w = workloads.Workload("parity", d, Bd, kb, m, kind, steps, seed=seed)
+    p0 = workloads.make_params(d, seed=7)
+    mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m)
+    state = mo.new_state("cuda")
+    p_gpu = p0.cuda()
+    ost = oracle.new_state(d, Bd, kb, m)
+    p_ref = p0.numpy().copy()
+    hyper = dict(lr=lr, beta1=b1, beta2=b2, eps=eps, wd=wd)
+    for t in range(1, steps + 1):
+        g = grads_fn(t) if grads_fn else workloads.make_grads(w, t)
+        g_gpu = g.cuda()
+        if use_step:
+            mo.step(p_gpu, g_gpu, state, t=t, seed=seed, **hyper)
+        else:
+            mhat = torch.zeros(d, device="cuda") if stats else None
+            vhat = torch.zeros(d, device="cuda") if stats else None
+            mo.select(g_gpu, state, t=t)
+            mo.apply(p_gpu, g_gpu, state, t=t, seed=seed, mhat=mhat, vhat=vhat, **hyper)
+        res = oracle.step(ost, p_ref, workloads.bf16_bits(g), t=t, seed=seed,
+                          want_stats=stats and not use_step, **hyper)
+        torch.cuda.synchronize()
+        what = f"(d={d} Bd={Bd} kb={kb} m={m})"
+        compare_state(mo, state, ost, t, d, m, kb, what)
+        compare_params(p_gpu, p_ref, lr, what + f" t={t}")
+        if stats and not use_step:
+            compare_stats(mhat, vhat, res, what + f" t={t}")
+    return mo, state, p_gpu
+
+
+def test_flat_2p20_twenty_steps():
+    """d = 2^20, N(0,1) bf16 gradients, B_d = 16384, k_b = 164, m = 10, 20 steps."""
+    run_parity(1 << 20, 16384, 164, 10, 20)
+
+
+def test_flat_2p20_through_mua_step():
+    """The production entry point (mua_step) gives the same state as select+apply."""
+    run_parity(1 << 20, 16384, 164, 10, 12, use_step=True, kind="t3")
+
+
+@pytest.mark.parametrize("d,Bd,kb,m,steps,kind", [
+    (5 * 2048 + 777, 2048, 21, 3, 8, "t3"),          # ragged odd-length last block
+    (3 * 8192 + 8, 8192, 82, 10, 12, "normal"),
+    (4 * 1022 + 301, 1022, 11, 4, 8, "normal"),      # B_d % 8 != 0: scalar path
+    (2 * 32766 + 1000, 32766, 328, 2, 4, "t3"),      # largest block, 1024 threads
+    (1000, 16384, 164, 10, 6, "normal"),             # d < B_d: one partial block
+    (1, 2, 1, 1, 4, "normal"),                       # d = 1
+    (37, 8, 1, 1, 6, "normal"),                      # k_b = 1, m = 1, tiny blocks
+    (3 * 16384, 16384, 164, 37, 40, "normal"),       # m = 37 (the m_max bound)
+    (64 * 33, 64, 64, 12, 12, "normal"),             # k_b = B_d: every entry kept
+])
+def test_shapes(d, Bd, kb, m, steps, kind):
+    run_parity(d, Bd, kb, m, steps, kind=kind)
+
+
+def test_weight_decay():
+    run_parity(3 * 4096 + 100, 4096, 41, 5, 6, wd=0.1, lr=1e-2)
+
+
+def test_ties_and_zero_blocks():
+    """Heavy ties (few distinct magnitudes) and an all-zero block."""
+    torch, _, workloads = _mods()
+    d, Bd = 6 * 1024, 1024
+    rng = np.random.default_rng(3)
+
+    def grads(t):
+        x = rng.choice([-2.0, -1.0, -0.5, 0.5, 1.0, 2.0], d).astype(np.float32)
+        x[Bd:2 * Bd] = 0.0
+        x[3 * Bd:4 * Bd] = 1.0
+        return workloads.grads_from_values(x)
+
+    run_parity(d, Bd, 11, 4, 8, grads_fn=grads)
+
+
+def test_adam_reduction_on_gpu():
+    """k_b = B_d, m >= T: the GPU step is Adam; the residual stays exactly 0."""
+    mo, state, _ = run_parity(4 * 250 + 16, 250 + 6, 256, 8, 8, lr=1e-2)
+    sb = state.cpu().numpy()
+    assert not state_view.codes(sb, mo.layout, mo.d).any()
+
+
+def test_nonfinite_sets_status():
+    torch, MicroAdam, workloads = _mods()
+    d = 4096
+    mo = MicroAdam(d, block_size=1024, k_per_block=11, window=2)
+    state = mo.new_state()
+    p = workloads.make_params(d).cuda()
+    g = torch.zeros(d, dtype=torch.bfloat16, device="cuda")
+    mo.step(p, g, state, lr=1e-3, beta1=.9, beta2=.999, eps=1e-8, wd=0., t=1, seed=1)
+    assert mo.status(state) == 0
+    g[1234] = float("nan")
+    mo.step(p, g, state, lr=1e-3, beta1=.9, beta2=.999, eps=1e-8, wd=0., t=2, seed=1)
+    assert mo.status(state) & 1
+    g[1234] = float("inf")
+    mo.step(p, g, state, lr=1e-3, beta1=.9, beta2=.999, eps=1e-8, wd=0., t=3, seed=1)
+    assert mo.status(state) & 1
+
+
+def test_deterministic_and_resumable():
+    """Two runs give identical bytes; a run saved after 5 steps and resumed from
+    a copy of its state matches the uninterrupted run bit for bit."""
+    torch, MicroAdam, workloads = _mods()
+    d, Bd, kb, m = 5 * 16384 + 3000, 16384, 164, 4
+    w = workloads.Workload("det", d, Bd, kb, m, "t3", 10)
+    hyper = dict(lr=1e-3, beta1=.9, beta2=.999, eps=1e-8, wd=0.)
+
+    def run(n, state=None, p=None, t0=1):
+        mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m)
+        state = mo.new_state() if state is None else state
+        p = workloads.make_params(d).cuda() if p is None else p
+        for t in range(t0, t0 + n):
+            mo.step(p, workloads.make_grads(w, t).cuda(), state, t=t, seed=9, **hyper)
+        torch.cuda.synchronize()
+        return state, p
+
+    s1, p1 = run(10)
+    s2, p2 = run(10)
+    assert torch.equal(s1, s2) and torch.equal(p1, p2)
+    s3, p3 = run(5)
+    saved_s, saved_p = s3.cpu().clone(), p3.cpu().clone()
+    s4, p4 = run(5, saved_s.cuda(), saved_p.cuda(), t0=6)
+    assert torch.equal(s4, s1) and torch.equal(p4, p1)
