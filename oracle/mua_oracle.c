@@ -24,8 +24,9 @@
  * notes):
  *  - Q is uniform 4-bit stochastic rounding between the 16 levels
  *    delta + c*(Delta-delta)/15, c = 0..15 (Lemma 1's (Delta-delta)/(2^b-1)
- *    level spacing), with c = min(15, floor(s + xi)), s = (x - delta) *
- *    (15/(Delta - delta)) and xi a 16-bit uniform draw in [0, 1).
+ *    level spacing), done at 16-bit resolution: with s the position in level
+ *    units and r a uniform 16-bit draw, c = min(15, floor((floor(2^16 s) + r)
+ *    / 2^16)), which rounds up with probability frac(s) to within 2^-16.
  *  - Top-k ties break to the lower index; a row lists its entries in
  *    ascending index order; V is the signed value rounded to bf16 (RNE).
  *  - m_hat = (1-beta1)/(1-beta1^t) * sum_r beta1^r V_r and likewise v_hat
@@ -129,19 +130,22 @@ void mua_oracle_dequantize(const uint8_t* codes, int64_t n, float delta, float D
     }
 }
 
-/* e = Q(x, delta, Delta): stochastic rounding of x onto the 16 levels.
- * base is the global index of x[0] (it selects the random draws). */
+/* e = Q(x, delta, Delta): stochastic rounding of x onto the 16 levels at
+ * 16-bit resolution. With s = (x - delta) * 15/(Delta - delta) in level units,
+ * S = floor(2^16 s) and r a uniform 16-bit draw, c = min(15, floor((S + r) / 2^16)):
+ * c = floor(s) + 1 with probability frac(S / 2^16), so E[c] = S / 2^16, within
+ * 2^-16 of s. base is the global index of x[0] (it selects the draws). */
 void mua_oracle_quantize(const float* x, int64_t n, int64_t base, float delta, float Delta,
                          int64_t t, uint64_t seed, uint8_t* codes) {
-    float inv = (Delta == delta) ? 0.0f : 15.0f / (Delta - delta);
+    float inv16 = (Delta == delta) ? 0.0f : (15.0f / (Delta - delta)) * 65536.0f;
     for (int64_t i = 0; i < n; ++i) {
-        float s = (x[i] - delta) * inv;
-        float xi = (float)mua_oracle_draw16(seed, t, base + i) * (1.0f / 65536.0f);
-        float y = s + xi;
-        unsigned c = 0;
-        if (y >= 1.0f) {
-            float f = floorf(y);
-            c = (f >= 15.0f) ? 15u : (unsigned)f;
+        float s16 = (x[i] - delta) * inv16;
+        uint32_t r = mua_oracle_draw16(seed, t, base + i);
+        unsigned c = 15u;
+        if (s16 >= 0.0f && s16 < 8388608.0f) {
+            uint32_t S = (uint32_t)floorf(s16);
+            uint32_t q = (S + r) >> 16;
+            c = (q > 15u) ? 15u : q;
         }
         put_code(codes, i, c);
     }

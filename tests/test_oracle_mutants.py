@@ -44,11 +44,14 @@ MUTANTS = {
         "float unit = (Delta - delta) / 15.0f;",
         "float unit = (Delta - delta) / 16.0f;"),
     "quantize_scale_16": (
-        "float inv = (Delta == delta) ? 0.0f : 15.0f / (Delta - delta);",
-        "float inv = (Delta == delta) ? 0.0f : 16.0f / (Delta - delta);"),
+        "float inv16 = (Delta == delta) ? 0.0f : (15.0f / (Delta - delta)) * 65536.0f;",
+        "float inv16 = (Delta == delta) ? 0.0f : (16.0f / (Delta - delta)) * 65536.0f;"),
     "quantize_round_to_nearest": (
-        "float y = s + xi;",
-        "float y = s + 0.5f;"),
+        "uint32_t q = (S + r) >> 16;",
+        "uint32_t q = (S + 32768u) >> 16;"),
+    "quantize_rounds_down_only": (
+        "uint32_t q = (S + r) >> 16;",
+        "uint32_t q = S >> 16;"),
     "philox_multiplier_swapped": (
         "uint64_t prod0 = (uint64_t)PHILOX_M0 * (uint64_t)c0;",
         "uint64_t prod0 = (uint64_t)PHILOX_M1 * (uint64_t)c0;"),
