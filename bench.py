@@ -249,16 +249,13 @@ def run_reference(args, rank, world):
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
-    from compressed_state_optimizer_b200 import MicroAdam, workloads as W
+    from compressed_state_optimizer_b200 import MicroAdam, sharding, workloads as W
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = get_workload(args.workload)
-    nb_total = -(-w.d // w.Bd)
-    b0 = nb_total * rank // world
-    b1 = nb_total * (rank + 1) // world
     mo = MicroAdam(w.d, block_size=w.Bd, k_per_block=w.kb, window=w.m,
-                   shard=None if world == 1 else (b0, b1 - b0))
+                   shard=None if world == 1 else sharding.shard_blocks(w.d, w.Bd, rank, world))
     d_loc, off = mo.d, mo.offset
     params = W.make_params(d_loc, seed=7 + rank, device=dev)
     grads = [W.make_grads(w, s, device=dev, start=off, length=d_loc) for s in (1, 2)]
@@ -270,9 +267,8 @@ def run_ours(args, rank, world, local_rank):
         if world == 1:
             mo.step(params, g, state, t=t, **hyper)
             return
-        mo.select(g, state, t=t)
-        o = mo.minmax_offset(t)
-        dist.all_reduce(state[o:o + 8].view(torch.int32), op=dist.ReduceOp.MAX)
+        mo.select(params, g, state, t=t, **hyper)
+        sharding.combine_minmax_(state, mo.minmax_offset(t))
         mo.apply(params, g, state, t=t, **hyper)
 
     def barrier():
@@ -298,11 +294,10 @@ def run_ours(args, rank, world, local_rank):
         t += 1
         g = grads[t % 2]
         ev[i][0].record(stream)
-        mo.select(g, state, t=t)
+        mo.select(params, g, state, t=t, **hyper)
         ev[i][1].record(stream)
         if world > 1:
-            o = mo.minmax_offset(t)
-            dist.all_reduce(state[o:o + 8].view(torch.int32), op=dist.ReduceOp.MAX)
+            sharding.combine_minmax_(state, mo.minmax_offset(t))
         mo.apply(params, g, state, t=t, **hyper)
         ev[i][2].record(stream)
     end.record(stream)

@@ -33,7 +33,9 @@ SIGNATURES = {
     "mua_state_bytes": (_i64, [_P]),
     "mua_state_layout": (ctypes.c_int, [_P, ctypes.POINTER(_i64)]),
     "mua_step": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P]),
-    "mua_select": (ctypes.c_int, [_P, _P, _P, _i64, _P]),
+    "mua_select": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P,
+                                  _P, _P]),
+    "mua_set_update_split": (ctypes.c_int, [_P, _i32]),
     "mua_minmax_offset": (_i64, [_P, _i64]),
     "mua_apply": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P,
                                  _P, _P]),
@@ -168,10 +170,26 @@ class MicroAdam:
                                   lr, beta1, beta2, eps, wd, t, seed, _stream_ptr(stream)),
                "mua_step")
 
-    def select(self, grads, state, *, t, stream=None):
-        self._check_tensors(None, grads, state)
-        _check(library().mua_select(self._h, grads.data_ptr(), state.data_ptr(), t,
-                                    _stream_ptr(stream)), "mua_select")
+    def select(self, params, grads, state, *, lr, beta1, beta2, eps, wd, t, seed, mhat=None,
+               vhat=None, stream=None):
+        """First half of step t (Top-k, window row, min/max partials, and the
+        parameter update of the blocks the select kernel owns)."""
+        self._half("mua_select", params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
+                   vhat, stream)
+
+    def set_update_split(self, split: int):
+        _check(library().mua_set_update_split(self._h, split), "mua_set_update_split")
+
+    def _half(self, name, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat, vhat,
+              stream):
+        self._check_tensors(params, grads, state)
+        for x in (mhat, vhat):
+            if x is not None:
+                assert x.is_cuda and x.numel() == self.d and x.is_contiguous()
+        fn = getattr(library(), name)
+        _check(fn(self._h, params.data_ptr(), grads.data_ptr(), state.data_ptr(), lr, beta1,
+                  beta2, eps, wd, t, seed, mhat.data_ptr() if mhat is not None else None,
+                  vhat.data_ptr() if vhat is not None else None, _stream_ptr(stream)), name)
 
     def minmax_offset(self, t: int) -> int:
         off = int(library().mua_minmax_offset(self._h, t))
@@ -181,15 +199,10 @@ class MicroAdam:
 
     def apply(self, params, grads, state, *, lr, beta1, beta2, eps, wd, t, seed, mhat=None,
               vhat=None, stream=None):
-        self._check_tensors(params, grads, state)
-        for x in (mhat, vhat):
-            if x is not None:
-                assert x.is_cuda and x.numel() == self.d and x.is_contiguous()
-        _check(library().mua_apply(self._h, params.data_ptr(), grads.data_ptr(),
-                                   state.data_ptr(), lr, beta1, beta2, eps, wd, t, seed,
-                                   mhat.data_ptr() if mhat is not None else None,
-                                   vhat.data_ptr() if vhat is not None else None,
-                                   _stream_ptr(stream)), "mua_apply")
+        """Second half of step t (4-bit quantization of the residual, and the
+        parameter update of the remaining blocks)."""
+        self._half("mua_apply", params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
+                   vhat, stream)
 
     def status(self, state, stream=None) -> int:
         out = ctypes.c_uint32()

@@ -5,9 +5,10 @@
 //
 // A handle holds geometry only. mua_step enqueues, on the caller's stream:
 //   1. an 8-byte memset of the (-delta_{t+1}, Delta_{t+1}) accumulator pair,
-//   2. the select kernel (one CTA per block),
+//   2. the select kernel (one CTA per block; also updates the parameters of
+//      the blocks with (j & 7) < update_split),
 //   3. the apply kernel (one CTA per block, reverse block order so the tail of
-//      the select kernel's reads is still in L2).
+//      the select kernel's reads is still in L2; updates the other blocks).
 // Everything the kernels need per step (beta^r weights, bias corrections,
 // Philox round keys) is computed here in fp64 and rounded once to fp32 /
 // uint32 before launch.
@@ -30,10 +31,16 @@ struct mua_ctx {
   int32_t threads;
   bool vec;             // 16-byte vector path usable (B_d % 8 == 0)
   int64_t off_codes, off_window, bytes;
-  uint32_t apply_smem;
+  uint32_t select_smem, apply_smem;
+  int32_t update_split;  // blocks with (j & 7) < split update in the select kernel
 };
 
 namespace {
+
+// Share of the blocks (in eighths) whose parameter update runs in the select
+// kernel: select does the arithmetic-heavy Top-k, apply the Philox codec; the
+// update is HBM traffic, placed to balance the two.
+constexpr int32_t kDefaultUpdateSplit = 4;
 
 thread_local char g_cuda_err[256] = "no CUDA error";
 
@@ -86,7 +93,9 @@ int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
   h->off_codes = 256;
   h->off_window = h->off_codes + round_up((h->d + 1) / 2, 256);
   h->bytes = h->off_window + 4 * block_count * (int64_t)m * kp;
+  h->select_smem = mua::select_smem_bytes(h->threads, Bd, kp, m);
   h->apply_smem = mua::apply_smem_bytes(h->threads, Bd, kp, m);
+  h->update_split = kDefaultUpdateSplit;
   *out = h;
   return MUA_OK;
 }
@@ -155,43 +164,21 @@ int64_t mua_minmax_offset(mua_t h, int64_t t) {
   return 4 * (int64_t)pair_word(t + 1);
 }
 
-int mua_select(mua_t h, const uint16_t* grads, void* state, int64_t t, void* stream) {
-  if (!h || !grads || !state || t < 1) return MUA_ERR_ARG;
-  if (!aligned16(grads) || !aligned16(state)) return MUA_ERR_ALIGN;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint8_t* st = static_cast<uint8_t*>(state);
-  mua::SelectArgs A;
-  A.g = geometry(h);
-  A.grads = grads;
-  A.codes = st + h->off_codes;
-  A.window = reinterpret_cast<uint32_t*>(st + h->off_window);
-  A.hdr = reinterpret_cast<uint32_t*>(st);
-  A.row = (int32_t)(t % h->m);
-  A.pair_cur = pair_word(t);
-  A.pair_next = pair_word(t + 1);
-  cudaError_t e = cudaMemsetAsync(A.hdr + A.pair_next, 0, 8, s);
-  if (e != cudaSuccess) return cuda_fail(e, "reset of the min/max pair");
-  e = mua::launch_select(A, h->threads, h->vec, s);
-  if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
-  return MUA_OK;
-}
-
-int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
-              float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
-              float* mhat, float* vhat, void* stream) {
+static int fill_args(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
+                     float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+                     float* mhat, float* vhat, mua::StepArgs* out) {
   if (!h || !params || !grads || !state) return MUA_ERR_ARG;
-  int rc = check_hyper(lr, beta1, beta2, eps, wd, t);
+  const int rc = check_hyper(lr, beta1, beta2, eps, wd, t);
   if (rc != MUA_OK) return rc;
   if (!aligned16(params) || !aligned16(grads) || !aligned16(state)) return MUA_ERR_ALIGN;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* st = static_cast<uint8_t*>(state);
-  mua::ApplyArgs A;
+  mua::StepArgs& A = *out;
   std::memset(&A, 0, sizeof A);
   A.g = geometry(h);
   A.params = params;
   A.grads = grads;
   A.codes = st + h->off_codes;
-  A.window = reinterpret_cast<const uint32_t*>(st + h->off_window);
+  A.window = reinterpret_cast<uint32_t*>(st + h->off_window);
   A.hdr = reinterpret_cast<uint32_t*>(st);
   A.mhat = mhat;
   A.vhat = vhat;
@@ -206,6 +193,7 @@ int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float 
   A.eps = eps;
   A.decay = (float)(1.0 - (double)lr * (double)wd);
   A.has_decay = (wd != 0.0f);
+  A.update_split = h->update_split;
   // Adam's bias correction of the unrolled sums [MicroAdam ¶1]:
   // m_hat = (1-beta1)/(1-beta1^t) * sum_r beta1^r V_r, likewise v_hat.
   A.f1 = (float)((1.0 - b1) / (1.0 - std::pow(b1, (double)t)));
@@ -215,29 +203,56 @@ int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float 
     A.w2[r] = (float)std::pow(b2, (double)r);
   }
   uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
-  for (int r = 0; r < 10; ++r) {
+  for (int r = 0; r < 10; ++r) {  // Philox4x32-10 round keys (Salmon et al.)
     A.keys[r][0] = k0;
     A.keys[r][1] = k1;
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
   }
-  A.reverse = 1;
-  A.smem_bytes = h->apply_smem;
-  const cudaError_t e = mua::launch_apply(A, h->threads, h->vec, s);
+  return MUA_OK;
+}
+
+int mua_select(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
+               float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+               float* mhat, float* vhat, void* stream) {
+  mua::StepArgs A;
+  const int rc = fill_args(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
+                           vhat, &A);
+  if (rc != MUA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(A.hdr + A.pair_next, 0, 8, s);
+  if (e != cudaSuccess) return cuda_fail(e, "reset of the min/max pair");
+  e = mua::launch_select(A, h->threads, h->vec, h->select_smem, s);
+  if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  return MUA_OK;
+}
+
+int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
+              float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+              float* mhat, float* vhat, void* stream) {
+  mua::StepArgs A;
+  const int rc = fill_args(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
+                           vhat, &A);
+  if (rc != MUA_OK) return rc;
+  const cudaError_t e =
+      mua::launch_apply(A, h->threads, h->vec, h->apply_smem, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "apply kernel launch");
   return MUA_OK;
 }
 
 int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float lr, float beta1,
              float beta2, float eps, float wd, int64_t t, uint64_t seed, void* stream) {
-  if (!h || !params || !grads || !state) return MUA_ERR_ARG;
-  int rc = check_hyper(lr, beta1, beta2, eps, wd, t);
-  if (rc != MUA_OK) return rc;
-  if (!aligned16(params) || !aligned16(grads) || !aligned16(state)) return MUA_ERR_ALIGN;
-  rc = mua_select(h, grads, state, t, stream);
+  int rc = mua_select(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, nullptr,
+                      nullptr, stream);
   if (rc != MUA_OK) return rc;
   return mua_apply(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, nullptr, nullptr,
                    stream);
+}
+
+int mua_set_update_split(mua_t h, int32_t split) {
+  if (!h || split < 0 || split > 8) return MUA_ERR_ARG;
+  h->update_split = split;
+  return MUA_OK;
 }
 
 int mua_get_status(mua_t h, const void* state, uint32_t* out, void* stream) {

@@ -1,5 +1,5 @@
-// Device-side building blocks shared by the two MicroAdam kernels
-// (mua_select.cu, mua_apply.cu) and the argument structs their launchers take.
+// Device-side building blocks of the two MicroAdam kernels (mua_select.cu,
+// mua_apply.cu) and the argument block both take.
 //
 // [MicroAdam ¶n] is paragraph n of "MicroAdam (Sparse-Gradient Adaptive
 // Optimization with Quantized Error Feedback)".
@@ -9,7 +9,11 @@
 // elements, chunk c starting at block-local index c*8*T + 8*tid. So every
 // chunk is one 16-byte load of bf16 gradients and one 4-byte load of packed
 // codes, a warp's loads are contiguous, and the local index order is
-// (c, tid, e) lexicographic, which the index-ordered scans below rely on.
+// (c, tid, e) lexicographic, which the index-ordered scans rely on.
+//
+// Exact conversions without the (quarter-rate) conversion unit:
+//   (float)c for 0 <= c < 2^23:  bits(0x4B000000 | c) - 2^23   (exact)
+//   floor(x) for 0 <= x < 2^23:  bits(x + 2^23 rounded toward zero) - 0x4B000000
 #pragma once
 
 #include <cstdint>
@@ -23,7 +27,10 @@ constexpr int kChunk = 8;
 constexpr int kChunks = kElemsPerThread / kChunk;
 constexpr int kMaxWindow = 64;            // m <= 64 (ages fit a 6-bit field)
 constexpr int kMaxWindowEntries = 16384;  // m * row_stride per block, on chip
+constexpr int kCandCap = 2048;            // select: on-chip candidate list
+constexpr int kHistBins = 2048;           // radix digit of 11 bits
 constexpr uint32_t kEmptySlot = 0x0000FFFFu;  // I = -1, V = +0
+constexpr uint32_t kNil = 0xFFFFFFFFu;
 
 // Header words (uint32) at the start of the state buffer.
 constexpr int kHdrPair0 = 0;   // (-delta, Delta) for even t
@@ -42,39 +49,32 @@ struct Geometry {
   int32_t last_len;    // length of the last block
 };
 
-struct SelectArgs {
-  Geometry g;
-  const uint16_t* grads;
-  const uint8_t* codes;
-  uint32_t* window;
-  uint32_t* hdr;
-  int32_t row;        // t mod m
-  int32_t pair_cur;   // header word of (-delta_t, Delta_t)
-  int32_t pair_next;  // header word of (-delta_{t+1}, Delta_{t+1})
-};
-
-struct ApplyArgs {
+// One argument block for both kernels of step t.
+struct StepArgs {
   Geometry g;
   float* params;
   const uint16_t* grads;
   uint8_t* codes;
-  const uint32_t* window;
+  uint32_t* window;
   uint32_t* hdr;
-  float* mhat;
+  float* mhat;        // optional outputs (NULL in production)
   float* vhat;
   int32_t row;        // t mod m
   int32_t rows;       // min(t, m)
-  int32_t pair_cur;
-  int32_t pair_next;
+  int32_t pair_cur;   // header word of (-delta_t, Delta_t)
+  int32_t pair_next;  // header word of (-delta_{t+1}, Delta_{t+1})
   uint32_t t_lo, t_hi;
   float lr, eps, decay, f1, f2;
   int32_t has_decay;
-  int32_t reverse;     // process blocks in reverse order
-  uint32_t smem_bytes;
-  float w1[kMaxWindow];          // fp32(beta1^r), r = age
-  float w2[kMaxWindow];          // fp32(beta2^r)
-  uint32_t keys[10][2];          // Philox round keys: seed + r*(W0, W1)
+  int32_t update_split;  // blocks with (j & 7) < update_split update in select
+  float w1[kMaxWindow];  // fp32(beta1^r), r = age
+  float w2[kMaxWindow];  // fp32(beta2^r)
+  uint32_t keys[10][2];  // Philox round keys: seed + r*(W0, W1)
 };
+
+__device__ __forceinline__ bool update_in_select(const StepArgs& A, int j) {
+  return (j & 7) < A.update_split;
+}
 
 // ---------------------------------------------------------------- memory
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
@@ -89,7 +89,6 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
   return v;
 }
 
-// Block-local element index of (chunk c, thread tid, element e).
 template <int T>
 __device__ __forceinline__ int elem_index(int c, int tid, int e) {
   return c * kChunk * T + kChunk * tid + e;
@@ -133,34 +132,44 @@ __device__ __forceinline__ uint32_t chunk_word(const uint4& v, int w) {
   return w == 0 ? v.x : (w == 1 ? v.y : (w == 2 ? v.z : v.w));
 }
 
-// a = f32(g) + (delta + f32(c) * unit), each operation rounded to nearest
-// with no contraction: stage (1) of [MicroAdam ¶1], bit-identical in both
-// kernels.
-__device__ __forceinline__ float dequant_add(uint32_t gbits16, uint32_t code, float delta,
-                                             float unit) {
-  const float gf = __uint_as_float(gbits16 << 16);
-  const float level = __fmul_rn(__uint2float_rn(code), unit);
-  return __fadd_rn(gf, __fadd_rn(delta, level));
+// fp32 bits of bf16 element e of a chunk.
+__device__ __forceinline__ uint32_t grad_bits(const uint4& v, int e) {
+  const uint32_t word = chunk_word(v, e >> 1);
+  return (e & 1) ? (word & 0xFFFF0000u) : (word << 16);
 }
 
-template <int T>
+// Q^{-1} levels delta + c * unit for c = 0..15, each computed as
+// fl(delta + fl(fl(c) * unit)) exactly as [MicroAdam ¶1]'s dequantization is
+// written; threads 0..15 fill the table, the caller synchronizes.
+__device__ __forceinline__ void fill_levels(float* lv, float delta, float unit) {
+  const int c = threadIdx.x;
+  if (c < 16) {
+    const float cf = __fsub_rn(__uint_as_float(0x4B000000u | (uint32_t)c), 8388608.0f);
+    lv[c] = __fadd_rn(delta, __fmul_rn(cf, unit));
+  }
+}
+
+// a = f32(g) + Q^{-1}(code) for every element of the thread (stage (1)).
 __device__ __forceinline__ void dequant_block(const uint4 (&gv)[kChunks],
-                                              const uint32_t (&cv)[kChunks], float delta,
-                                              float unit, float (&a)[kElemsPerThread]) {
+                                              const uint32_t (&cv)[kChunks], const float* lv,
+                                              uint32_t (&ab)[kElemsPerThread]) {
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
 #pragma unroll
     for (int e = 0; e < kChunk; ++e) {
-      const uint32_t word = chunk_word(gv[c], e >> 1);
-      const uint32_t gb = (e & 1) ? (word >> 16) : (word & 0xFFFFu);
-      const uint32_t code = (cv[c] >> (4 * e)) & 0xFu;
-      a[c * kChunk + e] = dequant_add(gb, code, delta, unit);
+      const float gf = __uint_as_float(grad_bits(gv[c], e));
+      const float lev = lv[(cv[c] >> (4 * e)) & 0xFu];
+      ab[c * kChunk + e] = __float_as_uint(__fadd_rn(gf, lev));
     }
   }
 }
 
-__device__ __forceinline__ uint32_t magnitude_key(float a) {
-  return __float_as_uint(a) & 0x7FFFFFFFu;
+// One 4-bit code of stage (4): c = min(15, floor((floor(2^16 s) + r) / 2^16)),
+// s16 = 2^16 s >= 0, r a 16-bit draw. Returns the code in bits 16..19 of the
+// result (bits 0..15 are scratch); the caller shifts it into place.
+__device__ __forceinline__ uint32_t quantize_code_hi(float s16, uint32_t r) {
+  const uint32_t big = __float_as_uint(__fadd_rz(s16, 8388608.0f));  // 0x4B000000 + floor
+  return min(big + r, 0x4B0FFFFFu);
 }
 
 // ---------------------------------------------------------------- scans
@@ -199,6 +208,25 @@ __device__ __forceinline__ V block_inclusive_scan(V x, V* scratch, V& total) {
   }
 }
 
+// Block max of a uint32 (ends with a barrier).
+template <int T>
+__device__ __forceinline__ uint32_t block_max_u32(uint32_t x, uint32_t* scratch) {
+  constexpr int NW = T / 32;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = max(x, __shfl_xor_sync(0xFFFFFFFFu, x, o));
+  if constexpr (NW == 1) {
+    return x;
+  } else {
+    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = x;
+    __syncthreads();
+    uint32_t r = scratch[0];
+#pragma unroll
+    for (int w = 1; w < NW; ++w) r = max(r, scratch[w]);
+    __syncthreads();
+    return r;
+  }
+}
+
 // ---------------------------------------------------------------- Philox
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) with precomputed round
 // keys. Counter (c0, c1, c2, c3); returns the four output words.
@@ -220,10 +248,129 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
   return make_uint4(c0, c1, c2, c3);
 }
 
+// ---------------------------------------------------------------- AdamStats + update
+// Shared-memory layout of block_update (dynamic, 4-byte words):
+//   mask[Wn] wpre[Wn] W[E] nxt[E] head[Ucap] scan[T/32]
+__host__ __device__ inline uint32_t update_smem_bytes(int threads, int Bd, int kp, int m) {
+  const int Wn = (Bd + 31) / 32;
+  const int E = m * kp;
+  const int Ucap = Bd < E ? Bd : E;
+  return (uint32_t)(4 * (2 * Wn + 2 * E + Ucap + threads / 32));
+}
+
+// Stage (6) for block j [MicroAdam ¶1]: m_hat = AdamStats(beta1, G) and
+// v_hat = AdamStats(beta2, G^2) over the block's window rows, then
+// p <- p*(1 - lr*wd) (dense, if wd != 0) and p <- p - lr*m_hat/(eps + sqrt(v_hat))
+// on the window's index union. The rows are staged in shared memory; a
+// bitmask + popcount prefix ranks the union; the entries of one index are
+// linked into a list and summed by one thread, oldest row first, so the result
+// does not depend on thread timing. Called by all T threads, after a barrier.
+template <int T>
+__device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t start, int L,
+                                             uint8_t* smem, const float* s_w1,
+                                             const float* s_w2) {
+  const int tid = threadIdx.x;
+  const Geometry& G = A.g;
+  const int Wn = (G.Bd + 31) >> 5;
+  const int E = G.m * G.kp;
+  const int Ucap = min(G.Bd, E);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* wpre = mask + Wn;
+  uint32_t* W = wpre + Wn;
+  uint32_t* nxt = W + E;
+  uint32_t* head = nxt + E;
+  uint32_t* scan = head + Ucap;
+
+  for (int w = tid; w < Wn; w += T) mask[w] = 0u;
+  for (int u = tid; u < Ucap; u += T) head[u] = kNil;
+  __syncthreads();
+
+  // Rows of steps t, t-1, ..., t-rows+1 (age 0 = this step's row).
+  const uint32_t* wblk = A.window + (int64_t)j * G.m * G.kp;
+  const int staged = A.rows * G.kp;
+  for (int e = tid; e < staged; e += T) {
+    const int age = e / G.kp;
+    const int slot = e - age * G.kp;
+    int phys = A.row - age;
+    if (phys < 0) phys += G.m;
+    const uint32_t v = wblk[phys * G.kp + slot];
+    W[e] = v;
+    const uint32_t idx = v & 0xFFFFu;
+    if (idx < (uint32_t)L) atomicOr(&mask[idx >> 5], 1u << (idx & 31));  // 0xFFFF: empty
+  }
+  __syncthreads();
+
+  const uint32_t pc = (tid < Wn) ? (uint32_t)__popc(mask[tid]) : 0u;
+  uint32_t U;
+  const uint32_t incl = block_inclusive_scan<T, uint32_t>(pc, scan, U);
+  if (tid < Wn) wpre[tid] = incl - pc;
+  __syncthreads();
+
+  for (int e = tid; e < staged; e += T) {
+    const uint32_t idx = W[e] & 0xFFFFu;
+    if (idx >= (uint32_t)L) continue;
+    const uint32_t w = idx >> 5;
+    const uint32_t rank = wpre[w] + (uint32_t)__popc(mask[w] & ((1u << (idx & 31)) - 1u));
+    const uint32_t age = (uint32_t)(e / G.kp);
+    nxt[e] = atomicExch(&head[rank], (age << 16) | (uint32_t)e);
+  }
+  if (A.has_decay) {
+    float* pb = A.params + start;
+    for (int i = tid; i < L; i += T) pb[i] = __fmul_rn(pb[i], A.decay);
+  }
+  __syncthreads();
+
+  for (uint32_t r = tid; r < U; r += T) {
+    const uint32_t h = head[r];
+    float z1 = 0.0f, z2 = 0.0f;
+    uint32_t idx = 0u;
+    int prev = 1 << 30;
+    for (;;) {  // oldest remaining row first
+      int best = -1;
+      uint32_t bv = 0u;
+      for (uint32_t l = h; l != kNil; l = nxt[l & 0xFFFFu]) {
+        const int age = (int)(l >> 16);
+        if (age < prev && age > best) {
+          best = age;
+          bv = W[l & 0xFFFFu];
+        }
+      }
+      if (best < 0) break;
+      const float V = __uint_as_float(bv & 0xFFFF0000u);
+      z1 = __fadd_rn(z1, __fmul_rn(s_w1[best], V));
+      z2 = __fadd_rn(z2, __fmul_rn(s_w2[best], __fmul_rn(V, V)));
+      idx = bv & 0xFFFFu;
+      prev = best;
+    }
+    const float mh = __fmul_rn(A.f1, z1);
+    const float vh = __fmul_rn(A.f2, z2);
+    const float u = __fdiv_rn(mh, __fadd_rn(A.eps, __fsqrt_rn(vh)));
+    float* pp = A.params + start + idx;
+    *pp = __fsub_rn(*pp, __fmul_rn(A.lr, u));
+    if (A.mhat) A.mhat[start + idx] = mh;
+    if (A.vhat) A.vhat[start + idx] = vh;
+  }
+}
+
+// Copies the AdamStats weights into shared memory with constant indices (so
+// they stay in the kernel's parameter bank). Caller synchronizes.
+__device__ __forceinline__ void load_weights(const StepArgs& A, float* s_w1, float* s_w2) {
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int r = 0; r < kMaxWindow; ++r) {
+      s_w1[r] = A.w1[r];
+      s_w2[r] = A.w2[r];
+    }
+  }
+}
+
 // ---------------------------------------------------------------- launchers
 // Host-side launchers (defined next to their kernels). Return a cudaError_t.
-cudaError_t launch_select(const SelectArgs& args, int threads, bool vec, cudaStream_t stream);
-cudaError_t launch_apply(const ApplyArgs& args, int threads, bool vec, cudaStream_t stream);
+cudaError_t launch_select(const StepArgs& args, int threads, bool vec, uint32_t smem,
+                          cudaStream_t stream);
+cudaError_t launch_apply(const StepArgs& args, int threads, bool vec, uint32_t smem,
+                         cudaStream_t stream);
+uint32_t select_smem_bytes(int threads, int Bd, int kp, int m);
 uint32_t apply_smem_bytes(int threads, int Bd, int kp, int m);
 
 }  // namespace mua

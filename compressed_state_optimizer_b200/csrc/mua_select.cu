@@ -1,27 +1,39 @@
 // Stage kernel 1 of the MicroAdam step ([MicroAdam ¶1] = paragraph 1 of
 // "MicroAdam (Sparse-Gradient Adaptive Optimization with Quantized Error
-// Feedback)"): for one block of B_d parameters per CTA,
+// Feedback)"), one CTA per block of B_d parameters:
 //   a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t)      (in registers, never stored)
 //   (I_t, V_t) = Top-k of |a_t| (ties to the lower index), written in
 //   ascending index order to row t mod m of the window G,
 //   the residual (a_t with the selected entries zeroed) reduced to its block
 //   min/max and folded into the global (-delta_{t+1}, Delta_{t+1}) pair with
-//   one pair of integer atomics per CTA.
+//   one pair of integer atomics per CTA,
+//   and, for the blocks assigned to this kernel (j & 7 < update_split), the
+//   AdamStats update of the block's parameters (block_update), which needs the
+//   new row but not delta_{t+1}; that moves HBM traffic into this
+//   arithmetic-heavier kernel.
 //
-// Top-k is an exact MSB-first radix select on the 31-bit magnitude patterns
-// (digits of 11, 11 and 9 bits, shared-memory histograms), followed by one
-// index-ordered block scan that places the selected entries. HBM traffic per
-// parameter: 2 B gradient + 0.5 B codes read; per selected entry 4 B written.
+// Exact Top-k in two tiers:
+//  * candidate tier: a lower bound tau_lo for the k-th largest magnitude is
+//    estimated from one sample per thread (a high order statistic of the warps'
+//    top-2 samples, aiming at ~2.5k candidates); elements with |a| >= tau_lo
+//    are written, in index order, to a shared-memory list; an exact radix
+//    select on the list uses digits that start at the highest bit where tau_lo
+//    and the list maximum differ, so keys clustered in a narrow range (the
+//    usual case once the error feedback carries quantization noise) still
+//    spread over the histogram;
+//  * full tier, when the estimate fails (fewer than k or more than the list
+//    capacity): the same exact radix select on all register-held keys.
+// Both tiers produce identical results: the k largest keys, ties to the lower
+// index. HBM traffic per parameter: 2 B gradient + 0.5 B codes read; per
+// selected entry 4 B written; plus block_update's traffic for its blocks.
 #include "mua_kernels.cuh"
 
 namespace mua {
 namespace {
 
-constexpr int kHistBins = 2048;
-
-// Finds the digit bin holding the krem-th largest remaining key: the largest b
-// with (count of bins >= b) >= krem. Writes the bin and the count strictly
-// above it to s_res[0], s_res[1].
+// Digit bin holding the krem-th largest remaining key: the largest b with
+// (count of bins >= b) >= krem. Writes the bin and the count strictly above it
+// to s_res[0], s_res[1].
 template <int T>
 __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int krem,
                                          uint32_t* scan_scratch, uint32_t* s_res) {
@@ -47,45 +59,33 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int kr
   }
 }
 
-template <int T, bool VEC>
-__global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1)) mua_select_kernel(const SelectArgs A) {
-  __shared__ uint32_t hist[kHistBins];
-  __shared__ uint32_t scan32[T / 32];
-  __shared__ unsigned long long scan64[2][T / 32];
-  __shared__ uint32_t s_res[2];
-  __shared__ float s_min[T / 32], s_max[T / 32];
+struct SelectShared {
+  uint32_t scan32[32];
+  unsigned long long scan64[32];
+  uint32_t res[2];
+  uint32_t top[64];
+  uint32_t tau_lo;
+  float mn[32], mx[32];
+  float levels[16];
+  float w1[kMaxWindow], w2[kMaxWindow];
+};
 
-  const int tid = threadIdx.x;
-  const int j = blockIdx.x;
-  const Geometry& G = A.g;
-  const int64_t start = (int64_t)j * G.Bd;
-  const int L = (j == G.nb - 1) ? G.last_len : G.Bd;
-  const int k = (int)(((int64_t)L * G.kb + G.Bd - 1) / G.Bd);
-
-  uint4 gv[kChunks];
-  uint32_t cv[kChunks];
-  load_block<T, VEC>(A.grads, A.codes, start, L, tid, gv, cv);
-
-  // (1) a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t).
-  const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
-  const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
-  const float unit = __fdiv_rn(__fsub_rn(Delta, delta), 15.0f);
-  float af[kElemsPerThread];
-  dequant_block<T>(gv, cv, delta, unit, af);
-  // Only the bit patterns stay live; the magnitude key is ab & 0x7FFFFFFF and
-  // every radix digit below lies in bits 0..30, so it reads ab directly.
-  uint32_t ab[kElemsPerThread];
-#pragma unroll
-  for (int i = 0; i < kElemsPerThread; ++i) ab[i] = __float_as_uint(af[i]);
-  if (L < kElemsPerThread * T) {  // slots past the block's end hold +0
-#pragma unroll
-    for (int c = 0; c < kChunks; ++c)
-#pragma unroll
-      for (int e = 0; e < kChunk; ++e)
-        if (elem_index<T>(c, tid, e) >= L) ab[c * kChunk + e] = 0u;
+// Writes a selected entry to its row slot.
+__device__ __forceinline__ void put_entry(uint32_t* row, uint32_t pos, int k, uint32_t idx,
+                                          uint32_t abits) {
+  if (pos < (uint32_t)k) {
+    const uint32_t vb = __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(abits)));
+    row[pos] = (idx & 0xFFFFu) | (vb << 16);
   }
+}
 
-  // (2) exact radix select of the k-th largest magnitude key tau.
+// Exact radix select over the register-held keys of the whole block (full
+// tier). Writes the row and folds every non-selected value into rmin/rmax.
+template <int T>
+__device__ void select_full(const uint32_t (&ab)[kElemsPerThread], int k, uint32_t* hist,
+                            SelectShared& sh, uint32_t* row, uint32_t* hdr, float& rmin,
+                            float& rmax) {
+  const int tid = threadIdx.x;
   uint32_t prefix = 0u, pmask = 0u;
   int krem = k;
 #pragma unroll 1
@@ -93,34 +93,31 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1)) mua_select_kerne
     const int shift = pass == 0 ? 20 : (pass == 1 ? 9 : 0);
     const int nbins = pass == 2 ? 512 : kHistBins;
     for (int b = tid; b < nbins; b += T) hist[b] = 0u;
-    if (tid == 0) {
-      s_res[0] = 0u;
-      s_res[1] = 0u;
-    }
+    if (tid == 0) sh.res[0] = sh.res[1] = 0u;
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < kElemsPerThread; ++i) {
+      // digits lie in bits 0..30, so the sign bit never matters here
       if ((ab[i] & pmask) == prefix) atomicAdd(&hist[(ab[i] >> shift) & (nbins - 1)], 1u);
     }
     __syncthreads();
     if (pass == 0 && tid == 0) {
-      // Keys >= 0x7F800000 (bins 0x7F8..0x7FF) are +-inf or NaN.
-      uint32_t bad = 0;
+      uint32_t bad = 0;  // keys >= 0x7F800000 (bins 0x7F8..) are +-inf or NaN
       for (int b = 0x7F8; b < kHistBins; ++b) bad |= hist[b];
-      if (bad) atomicOr(&A.hdr[kHdrStatus], kStatusNonFinite);
+      if (bad) atomicOr(&hdr[kHdrStatus], kStatusNonFinite);
     }
-    find_bin<T>(hist, nbins, krem, scan32, s_res);
+    find_bin<T>(hist, nbins, krem, sh.scan32, sh.res);
     __syncthreads();
-    prefix |= s_res[0] << shift;
+    prefix |= sh.res[0] << shift;
     pmask |= (uint32_t)(nbins - 1) << shift;
-    krem -= (int)s_res[1];
+    krem -= (int)sh.res[1];
     __syncthreads();
   }
   const uint32_t tau = prefix;
-  const int need = krem;  // keys equal to tau to take, lowest indices first
+  const int need = krem;
 
-  // Index-ordered positions: per chunk, counts of keys > tau and == tau,
-  // packed in 16-bit fields (each field total <= 8*T <= 8192).
+  // Counts per chunk of keys > tau (bits 0..15 of each 32-bit half) and
+  // == tau, packed: field c of pg/pe holds chunk c (each total <= 8T <= 8192).
   unsigned long long pg = 0ull, pe = 0ull;
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
@@ -135,12 +132,8 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1)) mua_select_kerne
     pe |= (unsigned long long)ne << (16 * c);
   }
   unsigned long long tg, te;
-  const unsigned long long xg = block_inclusive_scan<T, unsigned long long>(pg, scan64[0], tg) - pg;
-  const unsigned long long xe = block_inclusive_scan<T, unsigned long long>(pe, scan64[1], te) - pe;
-
-  // (2)+(3) write the selected entries; the residual keeps the rest.
-  uint32_t* row = A.window + ((int64_t)j * G.m + A.row) * G.kp;
-  float rmin = 0.0f, rmax = 0.0f;  // selected entries become +0
+  const unsigned long long xg = block_inclusive_scan<T, unsigned long long>(pg, sh.scan64, tg) - pg;
+  const unsigned long long xe = block_inclusive_scan<T, unsigned long long>(pe, sh.scan64, te) - pe;
   uint32_t base_g = 0, base_e = 0;
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
@@ -150,75 +143,288 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1)) mua_select_kerne
     base_e += (uint32_t)((te >> (16 * c)) & 0xFFFFu);
 #pragma unroll
     for (int e = 0; e < kChunk; ++e) {
-      const float v = __uint_as_float(ab[c * kChunk + e]);
-      const uint32_t key = ab[c * kChunk + e] & 0x7FFFFFFFu;
-      bool sel = false;
-      uint32_t pos = 0;
+      const uint32_t bits = ab[c * kChunk + e];
+      const uint32_t key = bits & 0x7FFFFFFFu;
       if (key > tau) {
-        sel = true;
-        pos = run_g + min(run_e, (uint32_t)need);
+        put_entry(row, run_g + min(run_e, (uint32_t)need), k, elem_index<T>(c, tid, e), bits);
         ++run_g;
-      } else if (key == tau) {
-        if (run_e < (uint32_t)need) {
-          sel = true;
-          pos = run_g + run_e;
-        }
+      } else if (key == tau && run_e < (uint32_t)need) {
+        put_entry(row, run_g + run_e, k, elem_index<T>(c, tid, e), bits);
         ++run_e;
-      }
-      if (sel && pos < (uint32_t)k) {
-        const uint32_t idx = (uint32_t)elem_index<T>(c, tid, e);
-        const uint32_t vb = __bfloat16_as_ushort(__float2bfloat16_rn(v));
-        row[pos] = (idx & 0xFFFFu) | (vb << 16);
       } else {
+        if (key == tau) ++run_e;
+        const float v = __uint_as_float(bits);
         rmin = fminf(rmin, v);
         rmax = fmaxf(rmax, v);
       }
     }
   }
+}
+
+// Exact radix select over the n-entry candidate list (index order), whose keys
+// all lie in [tau_lo, max]. Writes the row and folds the non-selected
+// candidates into rmin/rmax.
+template <int T>
+__device__ void select_list(const uint32_t* cab, const uint16_t* cidx, int n, int k,
+                            uint32_t tau_lo, uint32_t* hist, SelectShared& sh, uint32_t* row,
+                            uint32_t* hdr, float& rmin, float& rmax) {
+  const int tid = threadIdx.x;
+  const int q = (n + T - 1) / T;       // entries per thread, contiguous
+  const int i0 = min(n, tid * q), i1 = min(n, i0 + q);
+
+  uint32_t kmax = 0u;
+  for (int i = i0; i < i1; ++i) kmax = max(kmax, cab[i] & 0x7FFFFFFFu);
+  kmax = block_max_u32<T>(kmax, sh.scan32);
+  if (tid == 0 && kmax >= 0x7F800000u) atomicOr(&hdr[kHdrStatus], kStatusNonFinite);
+
+  uint32_t tau = tau_lo;
+  int need = k;
+  const uint32_t diff = kmax ^ tau_lo;
+  if (diff != 0u) {
+    int hi = 31 - __clz(diff);  // highest bit where candidates can differ
+    uint32_t pmask = (hi >= 30) ? 0u : ((0xFFFFFFFFu << (hi + 1)) & 0x7FFFFFFFu);
+    uint32_t prefix = tau_lo & pmask;
+    int krem = k;
+#pragma unroll 1
+    while (hi >= 0) {
+      const int width = min(11, hi + 1);
+      const int shift = hi + 1 - width;
+      const int nbins = 1 << width;
+      for (int b = tid; b < nbins; b += T) hist[b] = 0u;
+      if (tid == 0) sh.res[0] = sh.res[1] = 0u;
+      __syncthreads();
+      for (int i = i0; i < i1; ++i) {
+        const uint32_t key = cab[i] & 0x7FFFFFFFu;
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nbins - 1)], 1u);
+      }
+      __syncthreads();
+      find_bin<T>(hist, nbins, krem, sh.scan32, sh.res);
+      __syncthreads();
+      prefix |= sh.res[0] << shift;
+      pmask |= (uint32_t)(nbins - 1) << shift;
+      krem -= (int)sh.res[1];
+      hi = shift - 1;
+      __syncthreads();
+    }
+    tau = prefix;
+    need = krem;
+  }
+
+  uint32_t cg = 0, ce = 0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t key = cab[i] & 0x7FFFFFFFu;
+    cg += key > tau;
+    ce += key == tau;
+  }
+  uint32_t tot;
+  const uint32_t packed = cg | (ce << 16);  // n <= kCandCap < 2^16
+  const uint32_t x = block_inclusive_scan<T, uint32_t>(packed, sh.scan32, tot) - packed;
+  uint32_t run_g = x & 0xFFFFu, run_e = x >> 16;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t bits = cab[i];
+    const uint32_t key = bits & 0x7FFFFFFFu;
+    if (key > tau) {
+      put_entry(row, run_g + min(run_e, (uint32_t)need), k, cidx[i], bits);
+      ++run_g;
+    } else if (key == tau && run_e < (uint32_t)need) {
+      put_entry(row, run_g + run_e, k, cidx[i], bits);
+      ++run_e;
+    } else {
+      if (key == tau) ++run_e;
+      const float v = __uint_as_float(bits);
+      rmin = fminf(rmin, v);
+      rmax = fmaxf(rmax, v);
+    }
+  }
+}
+
+template <int T, bool VEC>
+__global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
+    mua_select_kernel(const StepArgs A) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  __shared__ SelectShared sh;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(dyn);
+  uint32_t* cab = hist + kHistBins;
+  uint16_t* cidx = reinterpret_cast<uint16_t*>(cab + kCandCap);
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, wid = tid >> 5;
+  constexpr int NW = T / 32;
+  const int j = blockIdx.x;
+  const Geometry& G = A.g;
+  const int64_t start = (int64_t)j * G.Bd;
+  const int L = (j == G.nb - 1) ? G.last_len : G.Bd;
+  const int k = (int)(((int64_t)L * G.kb + G.Bd - 1) / G.Bd);
+
+  uint4 gv[kChunks];
+  uint32_t cv[kChunks];
+  load_block<T, VEC>(A.grads, A.codes, start, L, tid, gv, cv);
+
+  // (1) a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t).
+  {
+    const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
+    const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
+    fill_levels(sh.levels, delta, __fdiv_rn(__fsub_rn(Delta, delta), 15.0f));
+  }
+  load_weights(A, sh.w1, sh.w2);
+  __syncthreads();
+  uint32_t ab[kElemsPerThread];
+  dequant_block(gv, cv, sh.levels, ab);
+  if (L < kElemsPerThread * T) {  // slots past the block's end hold +0
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e)
+        if (elem_index<T>(c, tid, e) >= L) ab[c * kChunk + e] = 0u;
+  }
+
+  uint32_t* row = A.window + ((int64_t)j * G.m + A.row) * G.kp;
+  float rmin = 0.0f, rmax = 0.0f;  // selected entries become +0
+
+  // (2) candidate tier: tau_lo from the warps' top-2 samples.
+  const int r_target = (5 * k + 63) / 64;  // ~2.5k candidates among 32T elements
+  bool listed = false;
+  if (8 * k <= L && r_target <= min(2 * NW, 32)) {
+    const uint32_t s = ab[0] & 0x7FFFFFFFu;  // one sample per thread, stride 8
+    uint32_t m1 = s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m1 = max(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
+    const int first = __ffs(__ballot_sync(0xFFFFFFFFu, s == m1)) - 1;
+    uint32_t m2 = (lane == first) ? 0u : s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m2 = max(m2, __shfl_xor_sync(0xFFFFFFFFu, m2, o));
+    if (lane == 0) {
+      sh.top[2 * wid] = m1;
+      sh.top[2 * wid + 1] = m2;
+    }
+    __syncthreads();
+    if (wid == 0) {
+      uint32_t v = (lane < 2 * NW) ? sh.top[lane] : 0u;
+      // bitonic sort, descending across the 32 lanes
+#pragma unroll
+      for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+          const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
+          const bool up = ((lane & size) == 0);
+          const bool lower = ((lane & stride) == 0);
+          v = (lower == up) ? max(v, o) : min(v, o);
+        }
+      }
+      const uint32_t tl = __shfl_sync(0xFFFFFFFFu, v, r_target - 1);
+      if (lane == 0) sh.tau_lo = tl;
+    }
+    __syncthreads();
+    const uint32_t tau_lo = sh.tau_lo;
+
+    // Index-ordered positions of the candidates; the rest are residual.
+    unsigned long long pc = 0ull;
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) {
+      uint32_t cnt = 0;
+#pragma unroll
+      for (int e = 0; e < kChunk; ++e) {
+        const uint32_t bits = ab[c * kChunk + e];
+        const bool cand = (bits & 0x7FFFFFFFu) >= tau_lo;
+        cnt += cand;
+        const float v = cand ? 0.0f : __uint_as_float(bits);
+        rmin = fminf(rmin, v);
+        rmax = fmaxf(rmax, v);
+      }
+      pc |= (unsigned long long)cnt << (16 * c);
+    }
+    unsigned long long tot;
+    const unsigned long long x = block_inclusive_scan<T, unsigned long long>(pc, sh.scan64, tot) - pc;
+    int n = 0;
+#pragma unroll
+    for (int c = 0; c < kChunks; ++c) n += (int)((tot >> (16 * c)) & 0xFFFFu);
+    if (n >= k && n <= kCandCap) {
+      uint32_t base = 0;
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        uint32_t run = base + (uint32_t)((x >> (16 * c)) & 0xFFFFu);
+        base += (uint32_t)((tot >> (16 * c)) & 0xFFFFu);
+#pragma unroll
+        for (int e = 0; e < kChunk; ++e) {
+          const uint32_t bits = ab[c * kChunk + e];
+          if ((bits & 0x7FFFFFFFu) >= tau_lo) {
+            if (run < (uint32_t)kCandCap) {
+              cab[run] = bits;
+              cidx[run] = (uint16_t)elem_index<T>(c, tid, e);
+            }
+            ++run;
+          }
+        }
+      }
+      __syncthreads();
+      select_list<T>(cab, cidx, n, k, tau_lo, hist, sh, row, A.hdr, rmin, rmax);
+      listed = true;
+    } else {
+      rmin = rmax = 0.0f;
+    }
+  }
+  // (2) full tier.
+  if (!listed) select_full<T>(ab, k, hist, sh, row, A.hdr, rmin, rmax);
   for (int s = k + tid; s < G.kp; s += T) row[s] = kEmptySlot;
 
-  // (5 first half) block residual min/max -> global pair, as ordered uint32.
+  // (4, first half) block residual min/max -> global pair, as ordered uint32.
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     rmin = fminf(rmin, __shfl_xor_sync(0xFFFFFFFFu, rmin, o));
     rmax = fmaxf(rmax, __shfl_xor_sync(0xFFFFFFFFu, rmax, o));
   }
-  if ((tid & 31) == 0) {
-    s_min[tid >> 5] = rmin;
-    s_max[tid >> 5] = rmax;
+  if (lane == 0) {
+    sh.mn[wid] = rmin;
+    sh.mx[wid] = rmax;
   }
   __syncthreads();
   if (tid == 0) {
-    for (int w = 1; w < T / 32; ++w) {
-      rmin = fminf(rmin, s_min[w]);
-      rmax = fmaxf(rmax, s_max[w]);
+    for (int w = 1; w < NW; ++w) {
+      rmin = fminf(rmin, sh.mn[w]);
+      rmax = fmaxf(rmax, sh.mx[w]);
     }
     const float negmin = 0.0f - rmin;  // >= +0, canonical zero
     const float maxv = rmax + 0.0f;    // >= +0
     atomicMax(&A.hdr[A.pair_next], __float_as_uint(negmin));
     atomicMax(&A.hdr[A.pair_next + 1], __float_as_uint(maxv));
   }
+
+  // (6) for this kernel's share of the blocks; the row above is complete.
+  if (update_in_select(A, j)) {
+    __syncthreads();
+    block_update<T>(A, j, start, L, dyn, sh.w1, sh.w2);
+  }
 }
 
 template <int T>
-cudaError_t launch_t(const SelectArgs& args, bool vec, cudaStream_t stream) {
-  if (vec)
-    mua_select_kernel<T, true><<<args.g.nb, T, 0, stream>>>(args);
-  else
-    mua_select_kernel<T, false><<<args.g.nb, T, 0, stream>>>(args);
+cudaError_t launch_t(const StepArgs& args, bool vec, uint32_t smem, cudaStream_t stream) {
+  auto kern = vec ? mua_select_kernel<T, true> : mua_select_kernel<T, false>;
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<args.g.nb, T, smem, stream>>>(args);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_select(const SelectArgs& args, int threads, bool vec, cudaStream_t stream) {
+uint32_t select_smem_bytes(int threads, int Bd, int kp, int m) {
+  const uint32_t own = 4 * kHistBins + 6 * kCandCap;
+  const uint32_t upd = update_smem_bytes(threads, Bd, kp, m);
+  return own > upd ? own : upd;
+}
+
+cudaError_t launch_select(const StepArgs& args, int threads, bool vec, uint32_t smem,
+                          cudaStream_t stream) {
   switch (threads) {
-    case 32: return launch_t<32>(args, vec, stream);
-    case 64: return launch_t<64>(args, vec, stream);
-    case 128: return launch_t<128>(args, vec, stream);
-    case 256: return launch_t<256>(args, vec, stream);
-    case 512: return launch_t<512>(args, vec, stream);
-    case 1024: return launch_t<1024>(args, vec, stream);
+    case 32: return launch_t<32>(args, vec, smem, stream);
+    case 64: return launch_t<64>(args, vec, smem, stream);
+    case 128: return launch_t<128>(args, vec, smem, stream);
+    case 256: return launch_t<256>(args, vec, smem, stream);
+    case 512: return launch_t<512>(args, vec, smem, stream);
+    case 1024: return launch_t<1024>(args, vec, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }

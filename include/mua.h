@@ -113,7 +113,7 @@ int mua_state_layout(mua_t h, int64_t* out);
 
 /*
  * mua_step — one full MicroAdam step t [MicroAdam ¶1] on `stream`:
- * mua_select followed by mua_apply without statistics outputs.
+ * mua_select followed by mua_apply, without statistics outputs.
  *   params  device, fp32[d], updated in place
  *   grads   device, bf16[d] (raw 16-bit patterns), read only
  *   state   device, mua_state_bytes(h) bytes, updated in place
@@ -130,13 +130,18 @@ int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float l
              void* stream);
 
 /*
- * mua_select — stages (1)-(3) and (5) of step t [MicroAdam ¶1]: a_t from
- * grads and e_t, the per-block Top-k written to row t mod m of G, and the
- * per-block residual min/max folded into the (-delta_{t+1}, Delta_{t+1}) pair
- * of the header (reset first). Reads grads; writes the window row and the
- * header pair at byte offset mua_minmax_offset(h, t).
+ * mua_select — first half of step t [MicroAdam ¶1]: stages (1)-(3) and (5):
+ * a_t from grads and e_t, the per-block Top-k written to row t mod m of G,
+ * the per-block residual min/max folded into the (-delta_{t+1}, Delta_{t+1})
+ * pair of the header (reset first, see mua_minmax_offset), and stage (6), the
+ * AdamStats update of params, for the blocks this kernel owns (see
+ * mua_set_update_split). Arguments as mua_step; mhat / vhat as mua_apply.
+ * mua_select(t) and mua_apply(t) must be called in that order with identical
+ * arguments; a sharded caller all-reduces the header pair between them.
  */
-int mua_select(mua_t h, const uint16_t* grads, void* state, int64_t t, void* stream);
+int mua_select(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
+               float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+               float* mhat, float* vhat, void* stream);
 
 /*
  * mua_minmax_offset — byte offset in the state of the two fp32 words
@@ -147,16 +152,26 @@ int mua_select(mua_t h, const uint16_t* grads, void* state, int64_t t, void* str
 int64_t mua_minmax_offset(mua_t h, int64_t t);
 
 /*
- * mua_apply — stages (4) and (6) of step t after mua_select(t): quantizes the
- * residual into e_{t+1} with (delta_{t+1}, Delta_{t+1}) and applies the
- * AdamStats update to params. If mhat / vhat are non-NULL (device, fp32[d]),
- * m_hat and v_hat are also written at every index of the window's union
- * (other entries are left untouched), for testing and diagnostics.
- * Arguments and errors as mua_step.
+ * mua_apply — second half of step t after mua_select(t): stage (4), the
+ * quantization of the residual into e_{t+1} with (delta_{t+1}, Delta_{t+1}),
+ * and stage (6) for the blocks mua_select left. If mhat / vhat are non-NULL
+ * (device, fp32[d]), m_hat and v_hat are also written at every index of the
+ * window's union (other entries are left untouched) by whichever of the two
+ * calls updates that block, for testing and diagnostics. Arguments and errors
+ * as mua_step.
  */
 int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
               float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
               float* mhat, float* vhat, void* stream);
+
+/*
+ * mua_set_update_split — which kernel applies stage (6) to block j: mua_select
+ * when (j mod 8) < split, mua_apply otherwise; 0 <= split <= 8 (default 4).
+ * The results do not depend on it (each block is updated exactly once, by
+ * the same arithmetic); it only moves HBM traffic between the two kernels to
+ * balance them. Host only; MUA_ERR_ARG when out of range.
+ */
+int mua_set_update_split(mua_t h, int32_t split);
 
 /*
  * mua_get_status — copy the state's sticky status word (MUA_STATUS_* bits)

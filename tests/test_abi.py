@@ -133,7 +133,12 @@ def test_step_rejects_null_and_misaligned(mua):
     ok, bad = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1008)
     assert lib.mua_step(m._h, None, ok, ok, 1e-3, .9, .999, 1e-8, 0., 1, 1, None) == -1
     assert lib.mua_step(m._h, bad, ok, ok, 1e-3, .9, .999, 1e-8, 0., 1, 1, None) == -3
-    assert lib.mua_select(m._h, ok, bad, 1, None) == -3
+    assert lib.mua_select(m._h, ok, ok, bad, 1e-3, .9, .999, 1e-8, 0., 1, 1, None, None,
+                          None) == -3
+    assert lib.mua_apply(m._h, ok, ok, ok, 1e-3, .9, .999, 1e-8, 0., 0, 1, None, None,
+                         None) == -1
+    assert lib.mua_set_update_split(m._h, 9) == -1
+    assert lib.mua_set_update_split(m._h, 0) == 0
     assert lib.mua_step(None, ok, ok, ok, 1e-3, .9, .999, 1e-8, 0., 1, 1, None) == -1
     assert lib.mua_minmax_offset(m._h, 0) == -1
     assert lib.mua_minmax_offset(m._h, 1) in (0, 8)

@@ -62,11 +62,14 @@ def compare_stats(mhat, vhat, stats, what=""):
 
 
 def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0.9,
-               b2=0.999, eps=1e-8, wd=0.0, grads_fn=None, stats=True, use_step=False):
+               b2=0.999, eps=1e-8, wd=0.0, grads_fn=None, stats=True, use_step=False,
+               split=None):
     torch, MicroAdam, workloads = _mods()
     w = workloads.Workload("parity", d, Bd, kb, m, kind, steps, seed=seed)
     p0 = workloads.make_params(d, seed=7)
     mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m)
+    if split is not None:
+        mo.set_update_split(split)
     state = mo.new_state("cuda")
     p_gpu = p0.cuda()
     ost = oracle.new_state(d, Bd, kb, m)
@@ -80,7 +83,7 @@ def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0
         else:
             mhat = torch.zeros(d, device="cuda") if stats else None
             vhat = torch.zeros(d, device="cuda") if stats else None
-            mo.select(g_gpu, state, t=t)
+            mo.select(p_gpu, g_gpu, state, t=t, seed=seed, mhat=mhat, vhat=vhat, **hyper)
             mo.apply(p_gpu, g_gpu, state, t=t, seed=seed, mhat=mhat, vhat=vhat, **hyper)
         res = oracle.step(ost, p_ref, workloads.bf16_bits(g), t=t, seed=seed,
                           want_stats=stats and not use_step, **hyper)
@@ -93,9 +96,11 @@ def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0
     return mo, state, p_gpu
 
 
-def test_flat_2p20_twenty_steps():
-    """d = 2^20, N(0,1) bf16 gradients, B_d = 16384, k_b = 164, m = 10, 20 steps."""
-    run_parity(1 << 20, 16384, 164, 10, 20)
+@pytest.mark.parametrize("split", [4, 0, 8])
+def test_flat_2p20_twenty_steps(split):
+    """d = 2^20, N(0,1) bf16 gradients, B_d = 16384, k_b = 164, m = 10, 20 steps;
+    the parameter update in either kernel or shared between them."""
+    run_parity(1 << 20, 16384, 164, 10, 20, split=split)
 
 
 def test_flat_2p20_through_mua_step():
@@ -118,8 +123,9 @@ def test_shapes(d, Bd, kb, m, steps, kind):
     run_parity(d, Bd, kb, m, steps, kind=kind)
 
 
-def test_weight_decay():
-    run_parity(3 * 4096 + 100, 4096, 41, 5, 6, wd=0.1, lr=1e-2)
+@pytest.mark.parametrize("split", [4, 0, 8])
+def test_weight_decay(split):
+    run_parity(9 * 4096 + 100, 4096, 41, 5, 6, wd=0.1, lr=1e-2, split=split)
 
 
 def test_ties_and_zero_blocks():
