@@ -49,6 +49,8 @@ def parse():
                     help="llama2_7b | flat_134m | flat_1m | bert_base | flat_1g_m<m>")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--update-split", type=int, default=None,
+                    help="eighths of the blocks whose parameter update runs in the select kernel")
     ap.add_argument("--cpu-sample", type=int, default=1 << 23,
                     help="parameters in the oracle's bounded sample")
     return ap.parse_args()
@@ -256,6 +258,8 @@ def run_ours(args, rank, world, local_rank):
     w = get_workload(args.workload)
     mo = MicroAdam(w.d, block_size=w.Bd, k_per_block=w.kb, window=w.m,
                    shard=None if world == 1 else sharding.shard_blocks(w.d, w.Bd, rank, world))
+    if args.update_split is not None:
+        mo.set_update_split(args.update_split)
     d_loc, off = mo.d, mo.offset
     params = W.make_params(d_loc, seed=7 + rank, device=dev)
     grads = [W.make_grads(w, s, device=dev, start=off, length=d_loc) for s in (1, 2)]

@@ -194,6 +194,8 @@ static int fill_args(mua_t h, float* params, const uint16_t* grads, void* state,
   A.decay = (float)(1.0 - (double)lr * (double)wd);
   A.has_decay = (wd != 0.0f);
   A.update_split = h->update_split;
+  // Exact for e < 2^16: (2^32 mod kp) < kp and e * kp < 2^31 keep the error below 1/kp.
+  A.kp_recip = (uint32_t)(((1ull << 32) + (uint64_t)h->kp - 1) / (uint64_t)h->kp);
   // Adam's bias correction of the unrolled sums [MicroAdam ¶1]:
   // m_hat = (1-beta1)/(1-beta1^t) * sum_r beta1^r V_r, likewise v_hat.
   A.f1 = (float)((1.0 - b1) / (1.0 - std::pow(b1, (double)t)));

@@ -28,6 +28,7 @@ constexpr int kChunks = kElemsPerThread / kChunk;
 constexpr int kMaxWindow = 64;            // m <= 64 (ages fit a 6-bit field)
 constexpr int kMaxWindowEntries = 16384;  // m * row_stride per block, on chip
 constexpr int kCandCap = 2048;            // select: on-chip candidate list
+constexpr int kSlots = 8;                 // select: candidate slots per thread
 constexpr int kHistBins = 2048;           // radix digit of 11 bits
 constexpr uint32_t kEmptySlot = 0x0000FFFFu;  // I = -1, V = +0
 constexpr uint32_t kNil = 0xFFFFFFFFu;
@@ -67,6 +68,7 @@ struct StepArgs {
   float lr, eps, decay, f1, f2;
   int32_t has_decay;
   int32_t update_split;  // blocks with (j & 7) < update_split update in select
+  uint32_t kp_recip;     // ceil(2^32 / kp): e / kp == __umulhi(e, kp_recip) for e < 2^16
   float w1[kMaxWindow];  // fp32(beta1^r), r = age
   float w2[kMaxWindow];  // fp32(beta2^r)
   uint32_t keys[10][2];  // Philox round keys: seed + r*(W0, W1)
@@ -208,6 +210,37 @@ __device__ __forceinline__ V block_inclusive_scan(V x, V* scratch, V& total) {
   }
 }
 
+// Inclusive block scan with a single barrier: every warp re-scans the warp
+// totals itself. `scratch` (T/32 entries) must not be written again before
+// the next barrier.
+template <int T, typename V>
+__device__ __forceinline__ V block_scan_1bar(V x, V* scratch, V& total) {
+  constexpr int NW = T / 32;
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const V y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if constexpr (NW == 1) {
+    total = __shfl_sync(0xFFFFFFFFu, x, 31);
+    return x;
+  } else {
+    if (lane == 31) scratch[wid] = x;
+    __syncthreads();
+    V w = (lane < NW) ? scratch[lane] : V(0);
+#pragma unroll
+    for (int o = 1; o < NW; o <<= 1) {
+      const V y = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += y;
+    }
+    const V off = __shfl_sync(0xFFFFFFFFu, w, (wid + 31) & 31);
+    total = __shfl_sync(0xFFFFFFFFu, w, NW - 1);
+    return x + (wid > 0 ? off : V(0));
+  }
+}
+
 // Block max of a uint32 (ends with a barrier).
 template <int T>
 __device__ __forceinline__ uint32_t block_max_u32(uint32_t x, uint32_t* scratch) {
@@ -288,15 +321,28 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   // Rows of steps t, t-1, ..., t-rows+1 (age 0 = this step's row).
   const uint32_t* wblk = A.window + (int64_t)j * G.m * G.kp;
   const int staged = A.rows * G.kp;
-  for (int e = tid; e < staged; e += T) {
-    const int age = e / G.kp;
-    const int slot = e - age * G.kp;
-    int phys = A.row - age;
-    if (phys < 0) phys += G.m;
-    const uint32_t v = wblk[phys * G.kp + slot];
-    W[e] = v;
-    const uint32_t idx = v & 0xFFFFu;
-    if (idx < (uint32_t)L) atomicOr(&mask[idx >> 5], 1u << (idx & 31));  // 0xFFFF: empty
+  for (int e0 = tid; e0 < staged; e0 += 4 * T) {
+    uint32_t v[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {  // loads first, then the bookkeeping
+      const int e = e0 + b * T;
+      v[b] = kEmptySlot;
+      if (e < staged) {
+        const int age = (int)__umulhi((uint32_t)e, A.kp_recip);
+        const int slot = e - age * G.kp;
+        int phys = A.row - age;
+        if (phys < 0) phys += G.m;
+        v[b] = wblk[phys * G.kp + slot];
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int e = e0 + b * T;
+      if (e >= staged) continue;
+      W[e] = v[b];
+      const uint32_t idx = v[b] & 0xFFFFu;
+      if (idx < (uint32_t)L) atomicOr(&mask[idx >> 5], 1u << (idx & 31));  // 0xFFFF: empty
+    }
   }
   __syncthreads();
 
@@ -311,7 +357,7 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
     if (idx >= (uint32_t)L) continue;
     const uint32_t w = idx >> 5;
     const uint32_t rank = wpre[w] + (uint32_t)__popc(mask[w] & ((1u << (idx & 31)) - 1u));
-    const uint32_t age = (uint32_t)(e / G.kp);
+    const uint32_t age = __umulhi((uint32_t)e, A.kp_recip);
     nxt[e] = atomicExch(&head[rank], (age << 16) | (uint32_t)e);
   }
   if (A.has_decay) {
@@ -320,35 +366,61 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   }
   __syncthreads();
 
-  for (uint32_t r = tid; r < U; r += T) {
-    const uint32_t h = head[r];
-    float z1 = 0.0f, z2 = 0.0f;
-    uint32_t idx = 0u;
-    int prev = 1 << 30;
-    for (;;) {  // oldest remaining row first
-      int best = -1;
-      uint32_t bv = 0u;
-      for (uint32_t l = h; l != kNil; l = nxt[l & 0xFFFFu]) {
-        const int age = (int)(l >> 16);
-        if (age < prev && age > best) {
-          best = age;
-          bv = W[l & 0xFFFFu];
+  // Up to kBatch union indices per thread per round: all parameter loads are
+  // issued before any store, so the read-modify-writes overlap in flight.
+  constexpr int kBatch = 4;
+  for (uint32_t r0 = 0; r0 < U; r0 += kBatch * T) {
+    uint32_t idx[kBatch];
+    float mh[kBatch], vh[kBatch], pv[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      const uint32_t r = r0 + (uint32_t)(b * T + tid);
+      idx[b] = kNil;
+      if (r >= U) continue;
+      const uint32_t h = head[r];
+      float z1, z2;
+      const uint32_t h2 = nxt[h & 0xFFFFu];
+      if (h2 == kNil) {  // the index is in one row only (the common case)
+        const uint32_t bv = W[h & 0xFFFFu];
+        const int age = (int)(h >> 16);
+        const float V = __uint_as_float(bv & 0xFFFF0000u);
+        z1 = __fmul_rn(s_w1[age], V);
+        z2 = __fmul_rn(s_w2[age], __fmul_rn(V, V));
+        idx[b] = bv & 0xFFFFu;
+      } else {  // several rows: sum oldest row first
+        z1 = 0.0f;
+        z2 = 0.0f;
+        idx[b] = W[h & 0xFFFFu] & 0xFFFFu;
+        int prev = 1 << 30;
+        for (;;) {
+          int best = -1;
+          uint32_t bv = 0u;
+          for (uint32_t l = h; l != kNil; l = nxt[l & 0xFFFFu]) {
+            const int age = (int)(l >> 16);
+            if (age < prev && age > best) {
+              best = age;
+              bv = W[l & 0xFFFFu];
+            }
+          }
+          if (best < 0) break;
+          const float V = __uint_as_float(bv & 0xFFFF0000u);
+          z1 = __fadd_rn(z1, __fmul_rn(s_w1[best], V));
+          z2 = __fadd_rn(z2, __fmul_rn(s_w2[best], __fmul_rn(V, V)));
+          prev = best;
         }
       }
-      if (best < 0) break;
-      const float V = __uint_as_float(bv & 0xFFFF0000u);
-      z1 = __fadd_rn(z1, __fmul_rn(s_w1[best], V));
-      z2 = __fadd_rn(z2, __fmul_rn(s_w2[best], __fmul_rn(V, V)));
-      idx = bv & 0xFFFFu;
-      prev = best;
+      mh[b] = __fmul_rn(A.f1, z1);
+      vh[b] = __fmul_rn(A.f2, z2);
+      pv[b] = A.params[start + idx[b]];
     }
-    const float mh = __fmul_rn(A.f1, z1);
-    const float vh = __fmul_rn(A.f2, z2);
-    const float u = __fdiv_rn(mh, __fadd_rn(A.eps, __fsqrt_rn(vh)));
-    float* pp = A.params + start + idx;
-    *pp = __fsub_rn(*pp, __fmul_rn(A.lr, u));
-    if (A.mhat) A.mhat[start + idx] = mh;
-    if (A.vhat) A.vhat[start + idx] = vh;
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b) {
+      if (idx[b] == kNil) continue;
+      const float u = __fdiv_rn(mh[b], __fadd_rn(A.eps, __fsqrt_rn(vh[b])));
+      A.params[start + idx[b]] = __fsub_rn(pv[b], __fmul_rn(A.lr, u));
+      if (A.mhat) A.mhat[start + idx[b]] = mh[b];
+      if (A.vhat) A.vhat[start + idx[b]] = vh[b];
+    }
   }
 }
 

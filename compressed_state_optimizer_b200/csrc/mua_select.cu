@@ -15,14 +15,16 @@
 // Exact Top-k in two tiers:
 //  * candidate tier: a lower bound tau_lo for the k-th largest magnitude is
 //    estimated from one sample per thread (a high order statistic of the warps'
-//    top-2 samples, aiming at ~2.5k candidates); elements with |a| >= tau_lo
-//    are written, in index order, to a shared-memory list; an exact radix
-//    select on the list uses digits that start at the highest bit where tau_lo
-//    and the list maximum differ, so keys clustered in a narrow range (the
-//    usual case once the error feedback carries quantization noise) still
-//    spread over the histogram;
+//    top-2 samples, aiming at a few times k candidates); elements with
+//    |a| >= tau_lo are written, in index order, to a shared-memory list; an
+//    exact radix select on the list uses digits that start at the highest bit
+//    where tau_lo and the block's largest magnitude differ, so keys clustered
+//    in a narrow range (the usual case once the error feedback carries
+//    quantization noise) still spread over the histogram. One pass usually
+//    isolates the k-th key; the whole tier takes about ten block barriers;
 //  * full tier, when the estimate fails (fewer than k or more than the list
-//    capacity): the same exact radix select on all register-held keys.
+//    capacity): the same exact radix select on all keys, re-reading the block
+//    from L2 on every pass.
 // Both tiers produce identical results: the k largest keys, ties to the lower
 // index. HBM traffic per parameter: 2 B gradient + 0.5 B codes read; per
 // selected entry 4 B written; plus block_update's traffic for its blocks.
@@ -61,8 +63,11 @@ __device__ __forceinline__ void find_bin(const uint32_t* hist, int nbins, int kr
 
 struct SelectShared {
   uint32_t scan32[32];
+  uint32_t scan32b[32];
+  uint32_t wsum[32];
+  uint32_t wmax[32];
   unsigned long long scan64[32];
-  uint32_t res[2];
+  uint32_t res[3];
   uint32_t top[64];
   uint32_t tau_lo;
   float mn[32], mx[32];
@@ -79,26 +84,66 @@ __device__ __forceinline__ void put_entry(uint32_t* row, uint32_t pos, int k, ui
   }
 }
 
-// Exact radix select over the register-held keys of the whole block (full
-// tier). Writes the row and folds every non-selected value into rmin/rmax.
-template <int T>
-__device__ void select_full(const uint32_t (&ab)[kElemsPerThread], int k, uint32_t* hist,
-                            SelectShared& sh, uint32_t* row, uint32_t* hdr, float& rmin,
-                            float& rmax) {
+// a_t of the 8 elements of chunk c of thread tid, re-read from global memory
+// (the block was just streamed, so this hits L2). Elements past L are +0.
+template <int T, bool VEC>
+__device__ __forceinline__ void chunk_values(const uint16_t* grads, const uint8_t* codes,
+                                             int64_t start, int L, int c, const float* lv,
+                                             uint32_t (&ab)[kChunk]) {
+  uint4 gv;
+  uint32_t cv;
+  const int tid = threadIdx.x;
+  const int e0 = elem_index<T>(c, tid, 0);
+  if (VEC && e0 + kChunk <= L) {
+    gv = *reinterpret_cast<const uint4*>(grads + start + e0);
+    cv = *reinterpret_cast<const uint32_t*>(codes + ((start + e0) >> 1));
+  } else {
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    uint32_t cw = 0u;
+    for (int e = 0; e < kChunk; ++e) {
+      if (e0 + e < L) {
+        const int64_t i = start + e0 + e;
+        const uint32_t byte = codes[i >> 1];
+        w[e >> 1] |= (uint32_t)grads[i] << (16 * (e & 1));
+        cw |= ((i & 1) ? (byte >> 4) : (byte & 0xFu)) << (4 * e);
+      }
+    }
+    gv = make_uint4(w[0], w[1], w[2], w[3]);
+    cv = cw;
+  }
+#pragma unroll
+  for (int e = 0; e < kChunk; ++e) {
+    const float a = __fadd_rn(__uint_as_float(grad_bits(gv, e)), lv[(cv >> (4 * e)) & 0xFu]);
+    ab[e] = (e0 + e < L) ? __float_as_uint(a) : 0u;
+  }
+}
+
+// Exact radix select over every key of the block (full tier, used when the
+// candidate estimate fails): digits of 11, 11 and 9 bits, each pass re-reading
+// the block from L2. Writes the row and folds every non-selected value into
+// rmin/rmax.
+// The arguments are plain pointers and values: a reference to the kernel's
+// parameter block would make every CTA copy that block to local memory.
+template <int T, bool VEC>
+__device__ __noinline__ void select_full(const uint16_t* grads, const uint8_t* codes,
+                                         uint32_t* hdr, int64_t start, int L, int k,
+                                         const float* lv, uint32_t* hist, SelectShared& sh,
+                                         uint32_t* row, float& rmin, float& rmax) {
   const int tid = threadIdx.x;
   uint32_t prefix = 0u, pmask = 0u;
   int krem = k;
-#pragma unroll 1
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = pass == 0 ? 20 : (pass == 1 ? 9 : 0);
     const int nbins = pass == 2 ? 512 : kHistBins;
     for (int b = tid; b < nbins; b += T) hist[b] = 0u;
     if (tid == 0) sh.res[0] = sh.res[1] = 0u;
     __syncthreads();
+    for (int c = 0; c < kChunks; ++c) {
+      uint32_t ab[kChunk];
+      chunk_values<T, VEC>(grads, codes, start, L, c, lv, ab);
 #pragma unroll
-    for (int i = 0; i < kElemsPerThread; ++i) {
-      // digits lie in bits 0..30, so the sign bit never matters here
-      if ((ab[i] & pmask) == prefix) atomicAdd(&hist[(ab[i] >> shift) & (nbins - 1)], 1u);
+      for (int e = 0; e < kChunk; ++e)  // digits lie in bits 0..30
+        if ((ab[e] & pmask) == prefix) atomicAdd(&hist[(ab[e] >> shift) & (nbins - 1)], 1u);
     }
     __syncthreads();
     if (pass == 0 && tid == 0) {
@@ -116,15 +161,16 @@ __device__ void select_full(const uint32_t (&ab)[kElemsPerThread], int k, uint32
   const uint32_t tau = prefix;
   const int need = krem;
 
-  // Counts per chunk of keys > tau (bits 0..15 of each 32-bit half) and
-  // == tau, packed: field c of pg/pe holds chunk c (each total <= 8T <= 8192).
+  // Counts per chunk of keys > tau and == tau, packed: 16-bit field c holds
+  // chunk c (each total <= 8T <= 8192).
   unsigned long long pg = 0ull, pe = 0ull;
-#pragma unroll
   for (int c = 0; c < kChunks; ++c) {
+    uint32_t ab[kChunk];
+    chunk_values<T, VEC>(grads, codes, start, L, c, lv, ab);
     uint32_t ng = 0, ne = 0;
 #pragma unroll
     for (int e = 0; e < kChunk; ++e) {
-      const uint32_t key = ab[c * kChunk + e] & 0x7FFFFFFFu;
+      const uint32_t key = ab[e] & 0x7FFFFFFFu;
       ng += key > tau;
       ne += key == tau;
     }
@@ -135,15 +181,16 @@ __device__ void select_full(const uint32_t (&ab)[kElemsPerThread], int k, uint32
   const unsigned long long xg = block_inclusive_scan<T, unsigned long long>(pg, sh.scan64, tg) - pg;
   const unsigned long long xe = block_inclusive_scan<T, unsigned long long>(pe, sh.scan64, te) - pe;
   uint32_t base_g = 0, base_e = 0;
-#pragma unroll
   for (int c = 0; c < kChunks; ++c) {
     uint32_t run_g = base_g + (uint32_t)((xg >> (16 * c)) & 0xFFFFu);
     uint32_t run_e = base_e + (uint32_t)((xe >> (16 * c)) & 0xFFFFu);
     base_g += (uint32_t)((tg >> (16 * c)) & 0xFFFFu);
     base_e += (uint32_t)((te >> (16 * c)) & 0xFFFFu);
+    uint32_t ab[kChunk];
+    chunk_values<T, VEC>(grads, codes, start, L, c, lv, ab);
 #pragma unroll
     for (int e = 0; e < kChunk; ++e) {
-      const uint32_t bits = ab[c * kChunk + e];
+      const uint32_t bits = ab[e];
       const uint32_t key = bits & 0x7FFFFFFFu;
       if (key > tau) {
         put_entry(row, run_g + min(run_e, (uint32_t)need), k, elem_index<T>(c, tid, e), bits);
@@ -161,80 +208,147 @@ __device__ void select_full(const uint32_t (&ab)[kElemsPerThread], int k, uint32
   }
 }
 
-// Exact radix select over the n-entry candidate list (index order), whose keys
-// all lie in [tau_lo, max]. Writes the row and folds the non-selected
-// candidates into rmin/rmax.
+// Exact radix select over the n-entry candidate list (index order); all keys lie
+// in [tau_lo, kmax]. hist (>= 2048 words) must be zero on entry. Writes the
+// row and folds the non-selected candidates into rmin/rmax.
 template <int T>
 __device__ void select_list(const uint32_t* cab, const uint16_t* cidx, int n, int k,
-                            uint32_t tau_lo, uint32_t* hist, SelectShared& sh, uint32_t* row,
-                            uint32_t* hdr, float& rmin, float& rmax) {
-  const int tid = threadIdx.x;
-  const int q = (n + T - 1) / T;       // entries per thread, contiguous
+                            uint32_t tau_lo, uint32_t kmax, uint32_t* hist, SelectShared& sh,
+                            uint32_t* row, float& rmin, float& rmax) {
+  constexpr int NW = T / 32;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int q = (n + T - 1) / T;  // entries per thread, contiguous
   const int i0 = min(n, tid * q), i1 = min(n, i0 + q);
 
-  uint32_t kmax = 0u;
-  for (int i = i0; i < i1; ++i) kmax = max(kmax, cab[i] & 0x7FFFFFFFu);
-  kmax = block_max_u32<T>(kmax, sh.scan32);
-  if (tid == 0 && kmax >= 0x7F800000u) atomicOr(&hdr[kHdrStatus], kStatusNonFinite);
-
-  uint32_t tau = tau_lo;
-  int need = k;
+  // mode 0: selected = key >= thr; mode 1: key > thr, or key == thr for the
+  // `need` lowest indices.
+  uint32_t thr = tau_lo;
+  int mode = 1, need = k;
   const uint32_t diff = kmax ^ tau_lo;
   if (diff != 0u) {
     int hi = 31 - __clz(diff);  // highest bit where candidates can differ
     uint32_t pmask = (hi >= 30) ? 0u : ((0xFFFFFFFFu << (hi + 1)) & 0x7FFFFFFFu);
     uint32_t prefix = tau_lo & pmask;
     int krem = k;
-#pragma unroll 1
+    bool first = true;
     while (hi >= 0) {
       const int width = min(11, hi + 1);
       const int shift = hi + 1 - width;
       const int nbins = 1 << width;
-      for (int b = tid; b < nbins; b += T) hist[b] = 0u;
-      if (tid == 0) sh.res[0] = sh.res[1] = 0u;
-      __syncthreads();
+      if (!first) {
+        for (int b = tid; b < nbins; b += T) hist[b] = 0u;
+        __syncthreads();
+      }
+      first = false;
       for (int i = i0; i < i1; ++i) {
         const uint32_t key = cab[i] & 0x7FFFFFFFu;
         if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nbins - 1)], 1u);
       }
       __syncthreads();
-      find_bin<T>(hist, nbins, krem, sh.scan32, sh.res);
+      // Warp w owns bins [w*per, (w+1)*per); lane l owns per/32 of them.
+      const int per = max(32, nbins / NW);
+      const int per_lane = per / 32;
+      const int b0 = wid * per + lane * per_lane;
+      uint32_t own = 0;
+      for (int b = 0; b < per_lane; ++b)
+        if (b0 + b < nbins) own += hist[b0 + b];
+      uint32_t incl = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) sh.wsum[wid] = incl;
       __syncthreads();
-      prefix |= sh.res[0] << shift;
+      uint32_t above = 0;  // keys in the bins of the warps above this one
+      for (int w = wid + 1; w < NW; ++w) above += sh.wsum[w];
+      uint32_t running = above + (__shfl_sync(0xFFFFFFFFu, incl, 31) - incl);
+      for (int b = per_lane - 1; b >= 0; --b) {
+        if (b0 + b >= nbins) continue;
+        const uint32_t h = hist[b0 + b];
+        if (running < (uint32_t)krem && running + h >= (uint32_t)krem) {
+          sh.res[0] = (uint32_t)(b0 + b);
+          sh.res[1] = running;
+          sh.res[2] = h;
+        }
+        running += h;
+      }
+      __syncthreads();
+      const uint32_t bin = sh.res[0], abv = sh.res[1], inbin = sh.res[2];
+      prefix |= bin << shift;
       pmask |= (uint32_t)(nbins - 1) << shift;
-      krem -= (int)sh.res[1];
+      krem -= (int)abv;
       hi = shift - 1;
-      __syncthreads();
+      if (inbin == (uint32_t)krem) {  // the whole bin is selected: exact threshold
+        thr = prefix;
+        mode = 0;
+        break;
+      }
+      __syncthreads();  // before the next pass clears the histogram
     }
-    tau = prefix;
-    need = krem;
+    if (mode == 1) {
+      thr = prefix;
+      need = krem;
+    }
   }
 
+  // Positions in index order: counts of (key > thr, key == thr) per thread.
   uint32_t cg = 0, ce = 0;
   for (int i = i0; i < i1; ++i) {
     const uint32_t key = cab[i] & 0x7FFFFFFFu;
-    cg += key > tau;
-    ce += key == tau;
+    if (mode == 0) {
+      cg += key >= thr;
+    } else {
+      cg += key > thr;
+      ce += key == thr;
+    }
   }
   uint32_t tot;
   const uint32_t packed = cg | (ce << 16);  // n <= kCandCap < 2^16
-  const uint32_t x = block_inclusive_scan<T, uint32_t>(packed, sh.scan32, tot) - packed;
+  const uint32_t x = block_scan_1bar<T, uint32_t>(packed, sh.scan32b, tot) - packed;
   uint32_t run_g = x & 0xFFFFu, run_e = x >> 16;
   for (int i = i0; i < i1; ++i) {
     const uint32_t bits = cab[i];
     const uint32_t key = bits & 0x7FFFFFFFu;
-    if (key > tau) {
+    const bool gt = (mode == 0) ? key >= thr : key > thr;
+    if (gt) {
       put_entry(row, run_g + min(run_e, (uint32_t)need), k, cidx[i], bits);
       ++run_g;
-    } else if (key == tau && run_e < (uint32_t)need) {
+    } else if (mode == 1 && key == thr && run_e < (uint32_t)need) {
       put_entry(row, run_g + run_e, k, cidx[i], bits);
       ++run_e;
     } else {
-      if (key == tau) ++run_e;
+      if (mode == 1 && key == thr) ++run_e;
       const float v = __uint_as_float(bits);
       rmin = fminf(rmin, v);
       rmax = fmaxf(rmax, v);
     }
+  }
+}
+
+// Folds a residual min/max over the whole CTA into the global pair.
+template <int T>
+__device__ __forceinline__ void block_minmax_to_global(float rmin, float rmax, SelectShared& sh,
+                                                       uint32_t* hdr, int pair_next) {
+  constexpr int NW = T / 32;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    rmin = fminf(rmin, __shfl_xor_sync(0xFFFFFFFFu, rmin, o));
+    rmax = fmaxf(rmax, __shfl_xor_sync(0xFFFFFFFFu, rmax, o));
+  }
+  if (lane == 0) {
+    sh.mn[wid] = rmin;
+    sh.mx[wid] = rmax;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < NW; ++w) {
+      rmin = fminf(rmin, sh.mn[w]);
+      rmax = fmaxf(rmax, sh.mx[w]);
+    }
+    atomicMax(&hdr[pair_next], __float_as_uint(0.0f - rmin));  // >= +0, canonical zero
+    atomicMax(&hdr[pair_next + 1], __float_as_uint(rmax + 0.0f));
   }
 }
 
@@ -243,6 +357,8 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
     mua_select_kernel(const StepArgs A) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ SelectShared sh;
+  // dynamic shared memory: radix histogram, candidate list (bits, indices);
+  // the parameter update reuses the same bytes afterwards.
   uint32_t* hist = reinterpret_cast<uint32_t*>(dyn);
   uint32_t* cab = hist + kHistBins;
   uint16_t* cidx = reinterpret_cast<uint16_t*>(cab + kCandCap);
@@ -260,13 +376,14 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
   uint32_t cv[kChunks];
   load_block<T, VEC>(A.grads, A.codes, start, L, tid, gv, cv);
 
-  // (1) a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t).
+  // (1) a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t), from the level table.
   {
     const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
     const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
     fill_levels(sh.levels, delta, __fdiv_rn(__fsub_rn(Delta, delta), 15.0f));
   }
   load_weights(A, sh.w1, sh.w2);
+  for (int b = tid; b < kHistBins; b += T) hist[b] = 0u;
   __syncthreads();
   uint32_t ab[kElemsPerThread];
   dequant_block(gv, cv, sh.levels, ab);
@@ -280,12 +397,14 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
 
   uint32_t* row = A.window + ((int64_t)j * G.m + A.row) * G.kp;
   float rmin = 0.0f, rmax = 0.0f;  // selected entries become +0
-
-  // (2) candidate tier: tau_lo from the warps' top-2 samples.
-  const int r_target = (5 * k + 63) / 64;  // ~2.5k candidates among 32T elements
   bool listed = false;
+
+  // (2) candidate tier. tau_lo: a high order statistic of the warps' top-2
+  // samples (one sample per thread, stride 8); every warp sorts the 2*NW
+  // values itself, so no broadcast barrier is needed.
+  const int r_target = (5 * k + 63) / 64;
   if (8 * k <= L && r_target <= min(2 * NW, 32)) {
-    const uint32_t s = ab[0] & 0x7FFFFFFFu;  // one sample per thread, stride 8
+    const uint32_t s = ab[0] & 0x7FFFFFFFu;
     uint32_t m1 = s;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m1 = max(m1, __shfl_xor_sync(0xFFFFFFFFu, m1, o));
@@ -298,46 +417,52 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
       sh.top[2 * wid + 1] = m2;
     }
     __syncthreads();
-    if (wid == 0) {
-      uint32_t v = (lane < 2 * NW) ? sh.top[lane] : 0u;
-      // bitonic sort, descending across the 32 lanes
+    uint32_t v = (lane < 2 * NW) ? sh.top[lane] : 0u;
 #pragma unroll
-      for (int size = 2; size <= 32; size <<= 1) {
+    for (int size = 2; size <= 32; size <<= 1) {  // bitonic sort, descending
 #pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-          const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
-          const bool up = ((lane & size) == 0);
-          const bool lower = ((lane & stride) == 0);
-          v = (lower == up) ? max(v, o) : min(v, o);
-        }
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, v, stride);
+        const bool up = ((lane & size) == 0);
+        const bool lower = ((lane & stride) == 0);
+        v = (lower == up) ? max(v, o) : min(v, o);
       }
-      const uint32_t tl = __shfl_sync(0xFFFFFFFFu, v, r_target - 1);
-      if (lane == 0) sh.tau_lo = tl;
     }
-    __syncthreads();
-    const uint32_t tau_lo = sh.tau_lo;
+    const uint32_t tau_lo = __shfl_sync(0xFFFFFFFFu, v, r_target - 1);
 
-    // Index-ordered positions of the candidates; the rest are residual.
+    // Counts of candidates per chunk (16-bit fields), residual min/max of the
+    // rest, and the largest key.
     unsigned long long pc = 0ull;
+    uint32_t kmax = 0u;
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) {
       uint32_t cnt = 0;
 #pragma unroll
       for (int e = 0; e < kChunk; ++e) {
         const uint32_t bits = ab[c * kChunk + e];
-        const bool cand = (bits & 0x7FFFFFFFu) >= tau_lo;
+        const uint32_t key = bits & 0x7FFFFFFFu;
+        const bool cand = key >= tau_lo;
         cnt += cand;
+        kmax = max(kmax, key);
         const float v = cand ? 0.0f : __uint_as_float(bits);
         rmin = fminf(rmin, v);
         rmax = fmaxf(rmax, v);
       }
       pc |= (unsigned long long)cnt << (16 * c);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+    if (lane == 0) sh.wmax[wid] = kmax;
     unsigned long long tot;
-    const unsigned long long x = block_inclusive_scan<T, unsigned long long>(pc, sh.scan64, tot) - pc;
+    const unsigned long long x = block_scan_1bar<T, unsigned long long>(pc, sh.scan64, tot) - pc;
+    kmax = (lane < NW) ? sh.wmax[lane] : 0u;  // written before the scan's barrier
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+    if (tid == 0 && kmax >= 0x7F800000u) atomicOr(&A.hdr[kHdrStatus], kStatusNonFinite);
     int n = 0;
 #pragma unroll
     for (int c = 0; c < kChunks; ++c) n += (int)((tot >> (16 * c)) & 0xFFFFu);
+
     if (n >= k && n <= kCandCap) {
       uint32_t base = 0;
 #pragma unroll
@@ -347,47 +472,28 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
 #pragma unroll
         for (int e = 0; e < kChunk; ++e) {
           const uint32_t bits = ab[c * kChunk + e];
-          if ((bits & 0x7FFFFFFFu) >= tau_lo) {
-            if (run < (uint32_t)kCandCap) {
-              cab[run] = bits;
-              cidx[run] = (uint16_t)elem_index<T>(c, tid, e);
-            }
-            ++run;
+          const bool cand = (bits & 0x7FFFFFFFu) >= tau_lo;
+          if (cand) {  // n <= kCandCap bounds run
+            cab[run] = bits;
+            cidx[run] = (uint16_t)elem_index<T>(c, tid, e);
           }
+          run += cand;
         }
       }
       __syncthreads();
-      select_list<T>(cab, cidx, n, k, tau_lo, hist, sh, row, A.hdr, rmin, rmax);
+      select_list<T>(cab, cidx, n, k, tau_lo, kmax, hist, sh, row, rmin, rmax);
       listed = true;
     } else {
       rmin = rmax = 0.0f;
     }
   }
-  // (2) full tier.
-  if (!listed) select_full<T>(ab, k, hist, sh, row, A.hdr, rmin, rmax);
-  for (int s = k + tid; s < G.kp; s += T) row[s] = kEmptySlot;
-
-  // (4, first half) block residual min/max -> global pair, as ordered uint32.
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    rmin = fminf(rmin, __shfl_xor_sync(0xFFFFFFFFu, rmin, o));
-    rmax = fmaxf(rmax, __shfl_xor_sync(0xFFFFFFFFu, rmax, o));
+  if (!listed) {
+    // (2) full tier.
+    select_full<T, VEC>(A.grads, A.codes, A.hdr, start, L, k, sh.levels, hist, sh, row, rmin,
+                        rmax);
   }
-  if (lane == 0) {
-    sh.mn[wid] = rmin;
-    sh.mx[wid] = rmax;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    for (int w = 1; w < NW; ++w) {
-      rmin = fminf(rmin, sh.mn[w]);
-      rmax = fmaxf(rmax, sh.mx[w]);
-    }
-    const float negmin = 0.0f - rmin;  // >= +0, canonical zero
-    const float maxv = rmax + 0.0f;    // >= +0
-    atomicMax(&A.hdr[A.pair_next], __float_as_uint(negmin));
-    atomicMax(&A.hdr[A.pair_next + 1], __float_as_uint(maxv));
-  }
+  for (int sl = k + tid; sl < G.kp; sl += T) row[sl] = kEmptySlot;
+  block_minmax_to_global<T>(rmin, rmax, sh, A.hdr, A.pair_next);
 
   // (6) for this kernel's share of the blocks; the row above is complete.
   if (update_in_select(A, j)) {
@@ -411,7 +517,7 @@ cudaError_t launch_t(const StepArgs& args, bool vec, uint32_t smem, cudaStream_t
 }  // namespace
 
 uint32_t select_smem_bytes(int threads, int Bd, int kp, int m) {
-  const uint32_t own = 4 * kHistBins + 6 * kCandCap;
+  const uint32_t own = 4u * kHistBins + 6u * kCandCap;
   const uint32_t upd = update_smem_bytes(threads, Bd, kp, m);
   return own > upd ? own : upd;
 }
