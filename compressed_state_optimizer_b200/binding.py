@@ -21,6 +21,7 @@ MUA_ERR_UNSUPPORTED = -2
 MUA_ERR_ALIGN = -3
 MUA_ERR_CUDA = -4
 MUA_STATUS_NONFINITE = 1
+MUA_STATUS_TIMEOUT = 2
 
 # Every symbol include/mua.h declares, with its ctypes signature.
 _P = ctypes.c_void_p
@@ -36,6 +37,7 @@ SIGNATURES = {
     "mua_select": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P,
                                   _P, _P]),
     "mua_set_update_split": (ctypes.c_int, [_P, _i32]),
+    "mua_set_pipelined": (ctypes.c_int, [_P, _i32]),
     "mua_minmax_offset": (_i64, [_P, _i64]),
     "mua_apply": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P,
                                  _P, _P]),
@@ -176,6 +178,9 @@ class MicroAdam:
         parameter update of the blocks the select kernel owns)."""
         self._half("mua_select", params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
                    vhat, stream)
+
+    def set_pipelined(self, enable: bool):
+        _check(library().mua_set_pipelined(self._h, int(bool(enable))), "mua_set_pipelined")
 
     def set_update_split(self, split: int):
         _check(library().mua_set_update_split(self._h, split), "mua_set_update_split")

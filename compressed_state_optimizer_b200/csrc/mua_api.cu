@@ -30,6 +30,7 @@ struct mua_ctx {
   int32_t last_len;
   int32_t threads;
   bool vec;             // 16-byte vector path usable (B_d % 8 == 0)
+  bool persistent;      // bulk-copy pipelined kernels usable (B_d % 32 == 0)
   int64_t off_codes, off_window, bytes;
   uint32_t select_smem, apply_smem;
   int32_t update_split;  // blocks with (j & 7) < split update in the select kernel
@@ -90,6 +91,7 @@ int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
   h->last_len = (int32_t)(h->d - (block_count - 1) * Bd);
   h->threads = pick_threads(Bd);
   h->vec = (Bd % 8) == 0;
+  h->persistent = false;  // mua_set_pipelined(h, 1) opts in
   h->off_codes = 256;
   h->off_window = h->off_codes + round_up((h->d + 1) / 2, 256);
   h->bytes = h->off_window + 4 * block_count * (int64_t)m * kp;
@@ -224,7 +226,7 @@ int mua_select(mua_t h, float* params, const uint16_t* grads, void* state, float
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(A.hdr + A.pair_next, 0, 8, s);
   if (e != cudaSuccess) return cuda_fail(e, "reset of the min/max pair");
-  e = mua::launch_select(A, h->threads, h->vec, h->select_smem, s);
+  e = mua::launch_select(A, h->threads, h->vec, h->persistent, h->select_smem, s);
   if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
   return MUA_OK;
 }
@@ -249,6 +251,12 @@ int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float l
   if (rc != MUA_OK) return rc;
   return mua_apply(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, nullptr, nullptr,
                    stream);
+}
+
+int mua_set_pipelined(mua_t h, int32_t enable) {
+  if (!h || (enable != 0 && enable != 1)) return MUA_ERR_ARG;
+  h->persistent = enable && (h->Bd % 32) == 0 && h->nb >= 2;
+  return MUA_OK;
 }
 
 int mua_set_update_split(mua_t h, int32_t split) {

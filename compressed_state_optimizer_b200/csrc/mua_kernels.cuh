@@ -38,6 +38,8 @@ constexpr int kHdrPair0 = 0;   // (-delta, Delta) for even t
 constexpr int kHdrPair1 = 2;   // (-delta, Delta) for odd t
 constexpr int kHdrStatus = 4;
 constexpr uint32_t kStatusNonFinite = 1u;
+constexpr uint32_t kStatusTimeout = 2u;   // a bounded wait gave up
+constexpr uint32_t kMaxWaitRounds = 1u << 22;  // try_wait rounds before giving up
 
 struct Geometry {
   int64_t d;           // elements of this handle
@@ -174,6 +176,63 @@ __device__ __forceinline__ uint32_t quantize_code_hi(float s16, uint32_t r) {
   return min(big + r, 0x4B0FFFFFu);
 }
 
+// ---------------------------------------------------------------- TMA bulk copies
+// 1-D bulk copies global -> shared (cp.async.bulk, no multicast) completing
+// on an mbarrier with a transaction count. Waits are bounded: after
+// kMaxWaitRounds unsuccessful try_wait rounds the caller gets false.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+  return ok != 0u;
+}
+// Bounded wait for the phase with the given parity to complete.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kMaxWaitRounds; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// The thread's 4 chunks of a block staged in shared memory (gradients as bf16
+// at g, codes at c; both start at the block's first element).
+template <int T>
+__device__ __forceinline__ void load_block_smem(const uint16_t* g, const uint8_t* c, int tid,
+                                                uint4 (&gv)[kChunks], uint32_t (&cv)[kChunks]) {
+#pragma unroll
+  for (int k = 0; k < kChunks; ++k) {
+    const int e0 = elem_index<T>(k, tid, 0);
+    gv[k] = *reinterpret_cast<const uint4*>(g + e0);
+    cv[k] = *reinterpret_cast<const uint32_t*>(c + (e0 >> 1));
+  }
+}
+
 // ---------------------------------------------------------------- scans
 // Inclusive block scan over T threads (T a multiple of 32). `scratch` needs
 // T/32 entries. Ends with a barrier so scratch can be reused at once.
@@ -281,14 +340,31 @@ __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_
   return make_uint4(c0, c1, c2, c3);
 }
 
+// Hardware approximations (PTX sqrt.approx / rcp.approx, relative error about
+// 2^-22): the update's fp32 result is compared at 1e-5, far above that.
+__device__ __forceinline__ float sqrt_approx(float x) {
+  float r;
+  asm("sqrt.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // ---------------------------------------------------------------- AdamStats + update
 // Shared-memory layout of block_update (dynamic, 4-byte words):
 //   mask[Wn] wpre[Wn] W[E] nxt[E] head[Ucap] scan[T/32]
+// Wn (mask words) is padded to a multiple of 4 so that W starts on a 16-byte
+// boundary (it is written with 16-byte stores).
+__host__ __device__ inline int mask_words_padded(int Bd) { return (((Bd + 31) / 32) + 3) & ~3; }
+
 __host__ __device__ inline uint32_t update_smem_bytes(int threads, int Bd, int kp, int m) {
-  const int Wn = (Bd + 31) / 32;
+  const int Wn = mask_words_padded(Bd);
   const int E = m * kp;
   const int Ucap = Bd < E ? Bd : E;
-  return (uint32_t)(4 * (2 * Wn + 2 * E + Ucap + threads / 32));
+  return (uint32_t)(4 * (2 * Wn + 2 * E + 2 * Ucap + threads / 32 + 1));
 }
 
 // Stage (6) for block j [MicroAdam ¶1]: m_hat = AdamStats(beta1, G) and
@@ -308,50 +384,57 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   const int E = G.m * G.kp;
   const int Ucap = min(G.Bd, E);
   uint32_t* mask = reinterpret_cast<uint32_t*>(smem);
-  uint32_t* wpre = mask + Wn;
-  uint32_t* W = wpre + Wn;
+  uint32_t* wpre = mask + mask_words_padded(G.Bd);
+  uint32_t* W = wpre + mask_words_padded(G.Bd);  // 16-byte aligned
   uint32_t* nxt = W + E;
   uint32_t* head = nxt + E;
-  uint32_t* scan = head + Ucap;
+  uint32_t* queue = head + Ucap;   // union ranks found in several rows
+  uint32_t* scan = queue + Ucap;
+  uint32_t* qcount = scan + T / 32;
 
   for (int w = tid; w < Wn; w += T) mask[w] = 0u;
   for (int u = tid; u < Ucap; u += T) head[u] = kNil;
+  if (tid == 0) *qcount = 0u;
   __syncthreads();
 
-  // Rows of steps t, t-1, ..., t-rows+1 (age 0 = this step's row).
+  // Rows of steps t, t-1, ..., t-rows+1 (age 0 = this step's row), staged 4
+  // entries (16 bytes) per load: rows are kp = 4q entries long and start on
+  // 16-byte boundaries, so a load never straddles two rows.
   const uint32_t* wblk = A.window + (int64_t)j * G.m * G.kp;
-  const int staged = A.rows * G.kp;
-  for (int e0 = tid; e0 < staged; e0 += 4 * T) {
-    uint32_t v[4];
+  const int staged4 = (A.rows * G.kp) >> 2;
+  for (int v0 = tid; v0 < staged4; v0 += 2 * T) {
+    uint4 v[2];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {  // loads first, then the bookkeeping
-      const int e = e0 + b * T;
-      v[b] = kEmptySlot;
-      if (e < staged) {
+    for (int b = 0; b < 2; ++b) {  // loads first, then the bookkeeping
+      const int e = 4 * (v0 + b * T);
+      v[b] = make_uint4(kEmptySlot, kEmptySlot, kEmptySlot, kEmptySlot);
+      if (v0 + b * T < staged4) {
         const int age = (int)__umulhi((uint32_t)e, A.kp_recip);
-        const int slot = e - age * G.kp;
         int phys = A.row - age;
         if (phys < 0) phys += G.m;
-        v[b] = wblk[phys * G.kp + slot];
+        v[b] = *reinterpret_cast<const uint4*>(wblk + phys * G.kp + (e - age * G.kp));
       }
     }
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int e = e0 + b * T;
-      if (e >= staged) continue;
-      W[e] = v[b];
-      const uint32_t idx = v[b] & 0xFFFFu;
-      if (idx < (uint32_t)L) atomicOr(&mask[idx >> 5], 1u << (idx & 31));  // 0xFFFF: empty
+    for (int b = 0; b < 2; ++b) {
+      if (v0 + b * T >= staged4) continue;
+      reinterpret_cast<uint4*>(W)[v0 + b * T] = v[b];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t idx = chunk_word(v[b], q) & 0xFFFFu;
+        if (idx < (uint32_t)L) atomicOr(&mask[idx >> 5], 1u << (idx & 31));  // 0xFFFF: empty
+      }
     }
   }
   __syncthreads();
 
   const uint32_t pc = (tid < Wn) ? (uint32_t)__popc(mask[tid]) : 0u;
   uint32_t U;
-  const uint32_t incl = block_inclusive_scan<T, uint32_t>(pc, scan, U);
+  const uint32_t incl = block_scan_1bar<T, uint32_t>(pc, scan, U);
   if (tid < Wn) wpre[tid] = incl - pc;
   __syncthreads();
 
+  const int staged = A.rows * G.kp;
   for (int e = tid; e < staged; e += T) {
     const uint32_t idx = W[e] & 0xFFFFu;
     if (idx >= (uint32_t)L) continue;
@@ -366,8 +449,12 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   }
   __syncthreads();
 
-  // Up to kBatch union indices per thread per round: all parameter loads are
-  // issued before any store, so the read-modify-writes overlap in flight.
+  // Pass 1, uniform across lanes: indices present in one row only (the common
+  // case); the others are queued. Up to kBatch indices per thread per round,
+  // all parameter loads issued before any store so the read-modify-writes
+  // overlap in flight. u = m_hat / (eps + sqrt(v_hat)) uses the hardware
+  // square root and reciprocal approximations (a few ulp, far inside the fp32
+  // update's error).
   constexpr int kBatch = 4;
   for (uint32_t r0 = 0; r0 < U; r0 += kBatch * T) {
     uint32_t idx[kBatch];
@@ -376,50 +463,65 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
     for (int b = 0; b < kBatch; ++b) {
       const uint32_t r = r0 + (uint32_t)(b * T + tid);
       idx[b] = kNil;
+      mh[b] = vh[b] = pv[b] = 0.0f;
       if (r >= U) continue;
       const uint32_t h = head[r];
-      float z1, z2;
-      const uint32_t h2 = nxt[h & 0xFFFFu];
-      if (h2 == kNil) {  // the index is in one row only (the common case)
-        const uint32_t bv = W[h & 0xFFFFu];
-        const int age = (int)(h >> 16);
-        const float V = __uint_as_float(bv & 0xFFFF0000u);
-        z1 = __fmul_rn(s_w1[age], V);
-        z2 = __fmul_rn(s_w2[age], __fmul_rn(V, V));
-        idx[b] = bv & 0xFFFFu;
-      } else {  // several rows: sum oldest row first
-        z1 = 0.0f;
-        z2 = 0.0f;
-        idx[b] = W[h & 0xFFFFu] & 0xFFFFu;
-        int prev = 1 << 30;
-        for (;;) {
-          int best = -1;
-          uint32_t bv = 0u;
-          for (uint32_t l = h; l != kNil; l = nxt[l & 0xFFFFu]) {
-            const int age = (int)(l >> 16);
-            if (age < prev && age > best) {
-              best = age;
-              bv = W[l & 0xFFFFu];
-            }
-          }
-          if (best < 0) break;
-          const float V = __uint_as_float(bv & 0xFFFF0000u);
-          z1 = __fadd_rn(z1, __fmul_rn(s_w1[best], V));
-          z2 = __fadd_rn(z2, __fmul_rn(s_w2[best], __fmul_rn(V, V)));
-          prev = best;
-        }
+      if (nxt[h & 0xFFFFu] != kNil) {
+        queue[atomicAdd(qcount, 1u)] = r;
+        continue;
       }
-      mh[b] = __fmul_rn(A.f1, z1);
-      vh[b] = __fmul_rn(A.f2, z2);
+      const uint32_t bv = W[h & 0xFFFFu];
+      const int age = (int)(h >> 16);
+      const float V = __uint_as_float(bv & 0xFFFF0000u);
+      idx[b] = bv & 0xFFFFu;
+      mh[b] = __fmul_rn(A.f1, __fmul_rn(s_w1[age], V));
+      vh[b] = __fmul_rn(A.f2, __fmul_rn(s_w2[age], __fmul_rn(V, V)));
       pv[b] = A.params[start + idx[b]];
     }
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
       if (idx[b] == kNil) continue;
-      const float u = __fdiv_rn(mh[b], __fadd_rn(A.eps, __fsqrt_rn(vh[b])));
+      const float u = __fmul_rn(mh[b], rcp_approx(__fadd_rn(A.eps, sqrt_approx(vh[b]))));
       A.params[start + idx[b]] = __fsub_rn(pv[b], __fmul_rn(A.lr, u));
-      if (A.mhat) A.mhat[start + idx[b]] = mh[b];
-      if (A.vhat) A.vhat[start + idx[b]] = vh[b];
+      if (A.mhat) {
+        A.mhat[start + idx[b]] = mh[b];
+        A.vhat[start + idx[b]] = vh[b];
+      }
+    }
+  }
+  __syncthreads();
+
+  // Pass 2: indices present in several rows, summed oldest row first.
+  const uint32_t nq = *qcount;
+  for (uint32_t qi = tid; qi < nq; qi += T) {
+    const uint32_t h = head[queue[qi]];
+    const uint32_t idx = W[h & 0xFFFFu] & 0xFFFFu;
+    float z1 = 0.0f, z2 = 0.0f;
+    int prev = 1 << 30;
+    for (;;) {
+      int best = -1;
+      uint32_t bv = 0u;
+      for (uint32_t l = h; l != kNil; l = nxt[l & 0xFFFFu]) {
+        const int age = (int)(l >> 16);
+        if (age < prev && age > best) {
+          best = age;
+          bv = W[l & 0xFFFFu];
+        }
+      }
+      if (best < 0) break;
+      const float V = __uint_as_float(bv & 0xFFFF0000u);
+      z1 = __fadd_rn(z1, __fmul_rn(s_w1[best], V));
+      z2 = __fadd_rn(z2, __fmul_rn(s_w2[best], __fmul_rn(V, V)));
+      prev = best;
+    }
+    const float mh = __fmul_rn(A.f1, z1);
+    const float vh = __fmul_rn(A.f2, z2);
+    const float u = __fmul_rn(mh, rcp_approx(__fadd_rn(A.eps, sqrt_approx(vh))));
+    float* pp = A.params + start + idx;
+    *pp = __fsub_rn(*pp, __fmul_rn(A.lr, u));
+    if (A.mhat) {
+      A.mhat[start + idx] = mh;
+      A.vhat[start + idx] = vh;
     }
   }
 }
@@ -438,8 +540,8 @@ __device__ __forceinline__ void load_weights(const StepArgs& A, float* s_w1, flo
 
 // ---------------------------------------------------------------- launchers
 // Host-side launchers (defined next to their kernels). Return a cudaError_t.
-cudaError_t launch_select(const StepArgs& args, int threads, bool vec, uint32_t smem,
-                          cudaStream_t stream);
+cudaError_t launch_select(const StepArgs& args, int threads, bool vec, bool persistent,
+                          uint32_t smem, cudaStream_t stream);
 cudaError_t launch_apply(const StepArgs& args, int threads, bool vec, uint32_t smem,
                          cudaStream_t stream);
 uint32_t select_smem_bytes(int threads, int Bd, int kp, int m);

@@ -28,6 +28,8 @@
 // Both tiers produce identical results: the k largest keys, ties to the lower
 // index. HBM traffic per parameter: 2 B gradient + 0.5 B codes read; per
 // selected entry 4 B written; plus block_update's traffic for its blocks.
+#include <algorithm>
+
 #include "mua_kernels.cuh"
 
 namespace mua {
@@ -67,6 +69,10 @@ struct SelectShared {
   uint32_t wsum[32];
   uint32_t wmax[32];
   unsigned long long scan64[32];
+  unsigned long long gkey[32];
+  uint32_t gcnt;
+  uint32_t mm[2];     // block residual (-min, max) bit patterns
+  uint32_t arrived;   // warps that have folded their min/max
   uint32_t res[3];
   uint32_t top[64];
   uint32_t tau_lo;
@@ -326,65 +332,60 @@ __device__ void select_list(const uint32_t* cab, const uint16_t* cidx, int n, in
   }
 }
 
-// Folds a residual min/max over the whole CTA into the global pair.
+// Folds a residual min/max over the whole CTA into the global pair without a
+// block barrier: every warp folds its partial into two shared words with
+// atomics (both values are >= +0 as -min and max, so their bit patterns order
+// like the values), and the last warp to arrive publishes them with one pair
+// of global atomics. sh.mm[] and sh.arrived must be zero on entry; the caller
+// resets them after a later barrier.
 template <int T>
 __device__ __forceinline__ void block_minmax_to_global(float rmin, float rmax, SelectShared& sh,
                                                        uint32_t* hdr, int pair_next) {
   constexpr int NW = T / 32;
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     rmin = fminf(rmin, __shfl_xor_sync(0xFFFFFFFFu, rmin, o));
     rmax = fmaxf(rmax, __shfl_xor_sync(0xFFFFFFFFu, rmax, o));
   }
   if (lane == 0) {
-    sh.mn[wid] = rmin;
-    sh.mx[wid] = rmax;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < NW; ++w) {
-      rmin = fminf(rmin, sh.mn[w]);
-      rmax = fmaxf(rmax, sh.mx[w]);
+    atomicMax(&sh.mm[0], __float_as_uint(0.0f - rmin));  // canonical +0
+    atomicMax(&sh.mm[1], __float_as_uint(rmax + 0.0f));
+    __threadfence_block();
+    if (atomicAdd(&sh.arrived, 1u) == NW - 1) {  // last warp: all partials are in
+      __threadfence_block();
+      atomicMax(&hdr[pair_next], atomicOr(&sh.mm[0], 0u));
+      atomicMax(&hdr[pair_next + 1], atomicOr(&sh.mm[1], 0u));
     }
-    atomicMax(&hdr[pair_next], __float_as_uint(0.0f - rmin));  // >= +0, canonical zero
-    atomicMax(&hdr[pair_next + 1], __float_as_uint(rmax + 0.0f));
   }
 }
 
+// Everything after the loads for block j: gv/cv hold the thread's 4 chunks;
+// sh.levels and sh.w1/w2 are filled; `work` is the dynamic shared-memory
+// scratch (histogram + candidate list, then block_update). Ends with the
+// block fully processed; the caller synchronizes before reusing `work`.
 template <int T, bool VEC>
-__global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
-    mua_select_kernel(const StepArgs A) {
-  extern __shared__ __align__(16) uint8_t dyn[];
-  __shared__ SelectShared sh;
-  // dynamic shared memory: radix histogram, candidate list (bits, indices);
-  // the parameter update reuses the same bytes afterwards.
-  uint32_t* hist = reinterpret_cast<uint32_t*>(dyn);
+__device__ __forceinline__ void select_block(const StepArgs& A, int j,
+                                             const uint4 (&gv)[kChunks],
+                                             const uint32_t (&cv)[kChunks], uint8_t* work,
+                                             SelectShared& sh) {
+  uint32_t* hist = reinterpret_cast<uint32_t*>(work);
   uint32_t* cab = hist + kHistBins;
   uint16_t* cidx = reinterpret_cast<uint16_t*>(cab + kCandCap);
 
   const int tid = threadIdx.x;
   const int lane = tid & 31, wid = tid >> 5;
   constexpr int NW = T / 32;
-  const int j = blockIdx.x;
   const Geometry& G = A.g;
   const int64_t start = (int64_t)j * G.Bd;
   const int L = (j == G.nb - 1) ? G.last_len : G.Bd;
   const int k = (int)(((int64_t)L * G.kb + G.Bd - 1) / G.Bd);
 
-  uint4 gv[kChunks];
-  uint32_t cv[kChunks];
-  load_block<T, VEC>(A.grads, A.codes, start, L, tid, gv, cv);
-
-  // (1) a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t), from the level table.
-  {
-    const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
-    const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
-    fill_levels(sh.levels, delta, __fdiv_rn(__fsub_rn(Delta, delta), 15.0f));
+  for (int b = tid; b < kHistBins; b += T) hist[b] = 0u;  // used after later barriers
+  if (tid == 0) {
+    sh.mm[0] = sh.mm[1] = 0u;
+    sh.arrived = 0u;
   }
-  load_weights(A, sh.w1, sh.w2);
-  for (int b = tid; b < kHistBins; b += T) hist[b] = 0u;
-  __syncthreads();
   uint32_t ab[kElemsPerThread];
   dequant_block(gv, cv, sh.levels, ab);
   if (L < kElemsPerThread * T) {  // slots past the block's end hold +0
@@ -498,12 +499,131 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
   // (6) for this kernel's share of the blocks; the row above is complete.
   if (update_in_select(A, j)) {
     __syncthreads();
-    block_update<T>(A, j, start, L, dyn, sh.w1, sh.w2);
+    block_update<T>(A, j, start, L, work, sh.w1, sh.w2);
+  }
+}
+
+// One CTA per block.
+template <int T, bool VEC>
+__global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
+    mua_select_kernel(const StepArgs A) {
+  extern __shared__ __align__(16) uint8_t dyn[];
+  __shared__ SelectShared sh;
+  const int j = blockIdx.x;
+  const int64_t start = (int64_t)j * A.g.Bd;
+  const int L = (j == A.g.nb - 1) ? A.g.last_len : A.g.Bd;
+  uint4 gv[kChunks];
+  uint32_t cv[kChunks];
+  load_block<T, VEC>(A.grads, A.codes, start, L, threadIdx.x, gv, cv);
+  {  // (1) the 16 levels of Q^{-1}(e_t, delta_t, Delta_t)
+    const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
+    const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
+    fill_levels(sh.levels, delta, __fdiv_rn(__fsub_rn(Delta, delta), 15.0f));
+  }
+  load_weights(A, sh.w1, sh.w2);
+  __syncthreads();
+  select_block<T, VEC>(A, j, gv, cv, dyn, sh);
+}
+
+// Persistent CTAs (B_d % 32 == 0): each CTA walks the blocks
+// j = blockIdx.x + i * gridDim.x. One shared-memory stage holds a block's
+// gradients and codes, filled by bulk copies (TMA): as soon as the threads
+// have moved block i into registers, the copy of block i+1 is issued, so it
+// lands while block i is processed. A ragged last block is read directly.
+// Shared memory: stage {bf16 g[B_d], codes[B_d/2]}, then `work`.
+template <int T>
+__global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
+    mua_select_persistent(const StepArgs A) {
+  extern __shared__ __align__(128) uint8_t dyn[];
+  __shared__ SelectShared sh;
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t s_fail;
+  const Geometry& G = A.g;
+  const int tid = threadIdx.x;
+  const uint32_t gbytes = 2u * (uint32_t)G.Bd, cbytes = (uint32_t)G.Bd / 2u;
+  const uint32_t stage_bytes = (gbytes + cbytes + 127u) & ~127u;
+  uint8_t* work = dyn + stage_bytes;
+  const int nfull = (G.last_len == G.Bd) ? G.nb : G.nb - 1;  // blocks fed by TMA
+  const int step = gridDim.x;
+
+  auto issue = [&](int jj) {  // one thread: stage <- block jj
+    fence_proxy_async();
+    mbar_expect_tx(&bar, gbytes + cbytes);
+    bulk_g2s(dyn, A.grads + (int64_t)jj * G.Bd, gbytes, &bar);
+    bulk_g2s(dyn + gbytes, A.codes + ((int64_t)jj * G.Bd >> 1), cbytes, &bar);
+  };
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    mbar_init_fence();
+    s_fail = 0u;
+  }
+  {  // (1) the 16 levels of Q^{-1}(e_t, delta_t, Delta_t)
+    const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
+    const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
+    fill_levels(sh.levels, delta, __fdiv_rn(__fsub_rn(Delta, delta), 15.0f));
+  }
+  load_weights(A, sh.w1, sh.w2);
+  __syncthreads();
+  if (tid == 0 && (int)blockIdx.x < nfull) issue(blockIdx.x);
+  uint32_t uses = 0;      // completed phases of `bar`
+  bool in_flight = (int)blockIdx.x < nfull;
+  for (int i = 0;; ++i) {
+    const int j = blockIdx.x + i * step;
+    if (j >= G.nb) break;
+    uint4 gv[kChunks];
+    uint32_t cv[kChunks];
+    if (j < nfull) {
+      if (!mbar_wait(&bar, uses & 1u)) atomicOr(&s_fail, 1u);
+      __syncthreads();
+      if (s_fail) break;
+      ++uses;
+      in_flight = false;
+      load_block_smem<T>(reinterpret_cast<const uint16_t*>(dyn), dyn + gbytes, tid, gv, cv);
+      __syncthreads();  // every thread has read the stage: refill it
+      const int jn = j + step;
+      if (jn < nfull) {
+        if (tid == 0) issue(jn);
+        in_flight = true;
+      }
+    } else {
+      load_block<T, true>(A.grads, A.codes, (int64_t)j * G.Bd, G.last_len, tid, gv, cv);
+    }
+    select_block<T, true>(A, j, gv, cv, work, sh);
+    __syncthreads();  // `work` is reused by the next block
+  }
+  if (s_fail) {
+    // A wait gave up: record it and give the copy still in flight a bounded
+    // chance to land before the CTA's shared memory is released.
+    if (tid == 0) {
+      atomicOr(&A.hdr[kHdrStatus], kStatusTimeout);
+      if (in_flight) (void)mbar_wait(&bar, uses & 1u);
+    }
+    __syncthreads();
   }
 }
 
 template <int T>
-cudaError_t launch_t(const StepArgs& args, bool vec, uint32_t smem, cudaStream_t stream) {
+cudaError_t launch_t(const StepArgs& args, bool vec, bool persistent, uint32_t smem,
+                     cudaStream_t stream) {
+  if (persistent) {
+    auto kern = mua_select_persistent<T>;
+    // must match the kernel: bf16 g[B_d] + codes[B_d/2], rounded up to 128 bytes
+    const uint32_t stage = (2u * (uint32_t)args.g.Bd + (uint32_t)args.g.Bd / 2u + 127u) & ~127u;
+    const uint32_t total = stage + smem;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)total);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, T, total)) !=
+        cudaSuccess)
+      return e;
+    const int grid = (int)std::min<int64_t>(args.g.nb, (int64_t)std::max(1, per_sm) * sms);
+    kern<<<grid, T, total, stream>>>(args);
+    return cudaGetLastError();
+  }
   auto kern = vec ? mua_select_kernel<T, true> : mua_select_kernel<T, false>;
   if (smem > 48 * 1024) {
     const cudaError_t e =
@@ -522,15 +642,15 @@ uint32_t select_smem_bytes(int threads, int Bd, int kp, int m) {
   return own > upd ? own : upd;
 }
 
-cudaError_t launch_select(const StepArgs& args, int threads, bool vec, uint32_t smem,
-                          cudaStream_t stream) {
+cudaError_t launch_select(const StepArgs& args, int threads, bool vec, bool persistent,
+                          uint32_t smem, cudaStream_t stream) {
   switch (threads) {
-    case 32: return launch_t<32>(args, vec, smem, stream);
-    case 64: return launch_t<64>(args, vec, smem, stream);
-    case 128: return launch_t<128>(args, vec, smem, stream);
-    case 256: return launch_t<256>(args, vec, smem, stream);
-    case 512: return launch_t<512>(args, vec, smem, stream);
-    case 1024: return launch_t<1024>(args, vec, smem, stream);
+    case 32: return launch_t<32>(args, vec, persistent, smem, stream);
+    case 64: return launch_t<64>(args, vec, persistent, smem, stream);
+    case 128: return launch_t<128>(args, vec, persistent, smem, stream);
+    case 256: return launch_t<256>(args, vec, persistent, smem, stream);
+    case 512: return launch_t<512>(args, vec, persistent, smem, stream);
+    case 1024: return launch_t<1024>(args, vec, persistent, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }

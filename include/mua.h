@@ -46,6 +46,8 @@ extern "C" {
 
 /* Status bits (sticky, in the state header). */
 #define MUA_STATUS_NONFINITE 1u  /* some a_t was NaN or +-inf; results unspecified  */
+#define MUA_STATUS_TIMEOUT 2u    /* a kernel's bounded wait for its own bulk copy gave
+                                    up; that step's results are unspecified           */
 
 /* Fields written by mua_state_layout(). */
 #define MUA_LAYOUT_HEADER 0      /* byte offset of the 256-byte scalar header        */
@@ -172,6 +174,15 @@ int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float 
  * balance them. Host only; MUA_ERR_ARG when out of range.
  */
 int mua_set_update_split(mua_t h, int32_t split);
+
+/*
+ * mua_set_pipelined — choose the kernel shape (0 or 1; default 0): 1 runs
+ * persistent CTAs that stream each next block into shared memory with bulk
+ * copies (used when B_d % 32 == 0 and there are at least 2 blocks), 0 runs one
+ * CTA per block. Results are identical either way. Host only; MUA_ERR_ARG
+ * when enable is not 0 or 1.
+ */
+int mua_set_pipelined(mua_t h, int32_t enable);
 
 /*
  * mua_get_status — copy the state's sticky status word (MUA_STATUS_* bits)
