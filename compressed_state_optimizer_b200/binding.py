@@ -37,7 +37,7 @@ SIGNATURES = {
     "mua_select": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P,
                                   _P, _P]),
     "mua_set_update_split": (ctypes.c_int, [_P, _i32]),
-    "mua_set_pipelined": (ctypes.c_int, [_P, _i32]),
+    "mua_set_select_variant": (ctypes.c_int, [_P, _i32]),
     "mua_minmax_offset": (_i64, [_P, _i64]),
     "mua_apply": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P,
                                  _P, _P]),
@@ -179,8 +179,9 @@ class MicroAdam:
         self._half("mua_select", params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
                    vhat, stream)
 
-    def set_pipelined(self, enable: bool):
-        _check(library().mua_set_pipelined(self._h, int(bool(enable))), "mua_set_pipelined")
+    def set_select_variant(self, variant: int):
+        """0: one warp per block (default); 1: one CTA per block; 2: persistent CTAs."""
+        _check(library().mua_set_select_variant(self._h, int(variant)), "mua_set_select_variant")
 
     def set_update_split(self, split: int):
         _check(library().mua_set_update_split(self._h, split), "mua_set_update_split")

@@ -31,6 +31,7 @@ struct mua_ctx {
   int32_t threads;
   bool vec;             // 16-byte vector path usable (B_d % 8 == 0)
   bool persistent;      // bulk-copy pipelined kernels usable (B_d % 32 == 0)
+  int32_t variant;      // select kernel: 0 warp per block, 1 CTA per block, 2 persistent CTAs
   int64_t off_codes, off_window, bytes;
   uint32_t select_smem, apply_smem;
   int32_t update_split;  // blocks with (j & 7) < split update in the select kernel
@@ -91,7 +92,8 @@ int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
   h->last_len = (int32_t)(h->d - (block_count - 1) * Bd);
   h->threads = pick_threads(Bd);
   h->vec = (Bd % 8) == 0;
-  h->persistent = false;  // mua_set_pipelined(h, 1) opts in
+  h->persistent = false;
+  h->variant = 0;
   h->off_codes = 256;
   h->off_window = h->off_codes + round_up((h->d + 1) / 2, 256);
   h->bytes = h->off_window + 4 * block_count * (int64_t)m * kp;
@@ -195,7 +197,8 @@ static int fill_args(mua_t h, float* params, const uint16_t* grads, void* state,
   A.eps = eps;
   A.decay = (float)(1.0 - (double)lr * (double)wd);
   A.has_decay = (wd != 0.0f);
-  A.update_split = h->update_split;
+  // The warp-per-block select does no parameter update: apply does them all.
+  A.update_split = (h->variant == 0) ? 0 : h->update_split;
   // Exact for e < 2^16: (2^32 mod kp) < kp and e * kp < 2^31 keep the error below 1/kp.
   A.kp_recip = (uint32_t)(((1ull << 32) + (uint64_t)h->kp - 1) / (uint64_t)h->kp);
   // Adam's bias correction of the unrolled sums [MicroAdam ¶1]:
@@ -226,7 +229,10 @@ int mua_select(mua_t h, float* params, const uint16_t* grads, void* state, float
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(A.hdr + A.pair_next, 0, 8, s);
   if (e != cudaSuccess) return cuda_fail(e, "reset of the min/max pair");
-  e = mua::launch_select(A, h->threads, h->vec, h->persistent, h->select_smem, s);
+  if (h->variant == 0)
+    e = mua::launch_select_warp(A, h->vec, s);
+  else
+    e = mua::launch_select(A, h->threads, h->vec, h->variant == 2, h->select_smem, s);
   if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
   return MUA_OK;
 }
@@ -253,9 +259,10 @@ int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float l
                    stream);
 }
 
-int mua_set_pipelined(mua_t h, int32_t enable) {
-  if (!h || (enable != 0 && enable != 1)) return MUA_ERR_ARG;
-  h->persistent = enable && (h->Bd % 32) == 0 && h->nb >= 2;
+int mua_set_select_variant(mua_t h, int32_t variant) {
+  if (!h || variant < 0 || variant > 2) return MUA_ERR_ARG;
+  if (variant == 2 && !((h->Bd % 32) == 0 && h->nb >= 2)) return MUA_ERR_UNSUPPORTED;
+  h->variant = variant;
   return MUA_OK;
 }
 

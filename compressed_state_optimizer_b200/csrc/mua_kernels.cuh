@@ -545,6 +545,8 @@ cudaError_t launch_select(const StepArgs& args, int threads, bool vec, bool pers
 cudaError_t launch_apply(const StepArgs& args, int threads, bool vec, uint32_t smem,
                          cudaStream_t stream);
 uint32_t select_smem_bytes(int threads, int Bd, int kp, int m);
+cudaError_t launch_select_warp(const StepArgs& args, bool vec, cudaStream_t stream);
+uint32_t select_warp_smem_bytes();
 uint32_t apply_smem_bytes(int threads, int Bd, int kp, int m);
 
 }  // namespace mua

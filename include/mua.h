@@ -176,13 +176,17 @@ int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float 
 int mua_set_update_split(mua_t h, int32_t split);
 
 /*
- * mua_set_pipelined — choose the kernel shape (0 or 1; default 0): 1 runs
- * persistent CTAs that stream each next block into shared memory with bulk
- * copies (used when B_d % 32 == 0 and there are at least 2 blocks), 0 runs one
- * CTA per block. Results are identical either way. Host only; MUA_ERR_ARG
- * when enable is not 0 or 1.
+ * mua_set_select_variant — the kernel shape of mua_select (results are
+ * identical for every variant):
+ *   0 (default) one warp per block, many blocks in flight per SM; all
+ *     parameter updates then run in mua_apply (mua_set_update_split ignored);
+ *   1 one CTA per block;
+ *   2 persistent CTAs streaming each next block into shared memory with
+ *     bulk copies (needs B_d % 32 == 0 and at least 2 blocks, else
+ *     MUA_ERR_UNSUPPORTED).
+ * Host only; MUA_ERR_ARG for other values.
  */
-int mua_set_pipelined(mua_t h, int32_t enable);
+int mua_set_select_variant(mua_t h, int32_t variant);
 
 /*
  * mua_get_status — copy the state's sticky status word (MUA_STATUS_* bits)

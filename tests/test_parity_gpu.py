@@ -63,11 +63,13 @@ def compare_stats(mhat, vhat, stats, what=""):
 
 def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0.9,
                b2=0.999, eps=1e-8, wd=0.0, grads_fn=None, stats=True, use_step=False,
-               split=None):
+               split=None, variant=None):
     torch, MicroAdam, workloads = _mods()
     w = workloads.Workload("parity", d, Bd, kb, m, kind, steps, seed=seed)
     p0 = workloads.make_params(d, seed=7)
     mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m)
+    if variant is not None:
+        mo.set_select_variant(variant)
     if split is not None:
         mo.set_update_split(split)
     state = mo.new_state("cuda")
@@ -96,11 +98,12 @@ def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0
     return mo, state, p_gpu
 
 
-@pytest.mark.parametrize("split", [4, 0, 8])
-def test_flat_2p20_twenty_steps(split):
-    """d = 2^20, N(0,1) bf16 gradients, B_d = 16384, k_b = 164, m = 10, 20 steps;
-    the parameter update in either kernel or shared between them."""
-    run_parity(1 << 20, 16384, 164, 10, 20, split=split)
+@pytest.mark.parametrize("variant,split", [(0, 0), (1, 4), (1, 0), (1, 8), (2, 4)])
+def test_flat_2p20_twenty_steps(variant, split):
+    """d = 2^20, N(0,1) bf16 gradients, B_d = 16384, k_b = 164, m = 10, 20 steps,
+    for every select kernel shape (warp per block, CTA per block, persistent
+    CTAs) and with the parameter update in either kernel or shared."""
+    run_parity(1 << 20, 16384, 164, 10, 20, split=split, variant=variant)
 
 
 def test_flat_2p20_through_mua_step():
@@ -123,9 +126,15 @@ def test_shapes(d, Bd, kb, m, steps, kind):
     run_parity(d, Bd, kb, m, steps, kind=kind)
 
 
-@pytest.mark.parametrize("split", [4, 0, 8])
-def test_weight_decay(split):
-    run_parity(9 * 4096 + 100, 4096, 41, 5, 6, wd=0.1, lr=1e-2, split=split)
+@pytest.mark.parametrize("variant,split", [(0, 0), (1, 4), (1, 8)])
+def test_weight_decay(variant, split):
+    run_parity(9 * 4096 + 100, 4096, 41, 5, 6, wd=0.1, lr=1e-2, split=split, variant=variant)
+
+
+@pytest.mark.parametrize("variant", [1, 2])
+def test_shapes_other_variants(variant):
+    """Ragged blocks and ties through the CTA-per-block and persistent shapes."""
+    run_parity(5 * 2048 + 777, 2048, 21, 3, 8, kind="t3", variant=variant, split=4)
 
 
 def test_ties_and_zero_blocks():
