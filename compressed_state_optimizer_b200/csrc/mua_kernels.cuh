@@ -26,9 +26,8 @@ constexpr int kElemsPerThread = 32;
 constexpr int kChunk = 8;
 constexpr int kChunks = kElemsPerThread / kChunk;
 constexpr int kMaxWindow = 64;            // m <= 64 (ages fit a 6-bit field)
-constexpr int kMaxWindowEntries = 16384;  // m * row_stride per block, on chip
+constexpr int kMaxWindowEntries = 15360;  // m * row_stride per block, on chip
 constexpr int kCandCap = 2048;            // select: on-chip candidate list
-constexpr int kSlots = 8;                 // select: candidate slots per thread
 constexpr int kHistBins = 2048;           // radix digit of 11 bits
 constexpr uint32_t kEmptySlot = 0x0000FFFFu;  // I = -1, V = +0
 constexpr uint32_t kNil = 0xFFFFFFFFu;
@@ -354,26 +353,32 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 
 // ---------------------------------------------------------------- AdamStats + update
-// Shared-memory layout of block_update (dynamic, 4-byte words):
-//   mask[Wn] wpre[Wn] W[E] nxt[E] head[Ucap] scan[T/32]
-// Wn (mask words) is padded to a multiple of 4 so that W starts on a 16-byte
-// boundary (it is written with 16-byte stores).
+// Shared-memory layout of block_update (dynamic):
+//   mask  u32[WnP]    bitmask of the window's index union (WnP = words padded to 4)
+//   wpre  u16[WnP8]   exclusive popcount prefix of mask (union rank of each word)
+//   W     u32[E]      staged rows, age-major; the index half becomes the union rank
+//   acc   float2[Ucap] (sum_r beta1^r V_r, sum_r beta2^r V_r^2) per union slot
+//   uidx  u16[Ucap]   block-relative index of each union slot
+//   scan  u32[T/32]   block scan scratch
+// Every region starts on a 16-byte boundary except uidx and scan (8 and 4).
 __host__ __device__ inline int mask_words_padded(int Bd) { return (((Bd + 31) / 32) + 3) & ~3; }
 
 __host__ __device__ inline uint32_t update_smem_bytes(int threads, int Bd, int kp, int m) {
-  const int Wn = mask_words_padded(Bd);
+  const int WnP = mask_words_padded(Bd);
   const int E = m * kp;
   const int Ucap = Bd < E ? Bd : E;
-  return (uint32_t)(4 * (2 * Wn + 2 * E + 2 * Ucap + threads / 32 + 1));
+  return (uint32_t)(4 * WnP + 2 * ((WnP + 7) & ~7) + 4 * E + 10 * Ucap + 4 * (threads / 32));
 }
 
 // Stage (6) for block j [MicroAdam ¶1]: m_hat = AdamStats(beta1, G) and
 // v_hat = AdamStats(beta2, G^2) over the block's window rows, then
 // p <- p*(1 - lr*wd) (dense, if wd != 0) and p <- p - lr*m_hat/(eps + sqrt(v_hat))
-// on the window's index union. The rows are staged in shared memory; a
-// bitmask + popcount prefix ranks the union; the entries of one index are
-// linked into a list and summed by one thread, oldest row first, so the result
-// does not depend on thread timing. Called by all T threads, after a barrier.
+// on the window's index union. The rows are staged in shared memory and a
+// bitmask + popcount prefix gives each index its union rank. The sums run one
+// row at a time, oldest row first: the indices of one row are distinct, so no
+// two threads touch one accumulator within a row, and every accumulator sees
+// its terms in the same order on every run. Called by all T threads, after a
+// barrier.
 template <int T>
 __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t start, int L,
                                              uint8_t* smem, const float* s_w1,
@@ -381,20 +386,17 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   const int tid = threadIdx.x;
   const Geometry& G = A.g;
   const int Wn = (G.Bd + 31) >> 5;
+  const int WnP = mask_words_padded(G.Bd);
   const int E = G.m * G.kp;
   const int Ucap = min(G.Bd, E);
   uint32_t* mask = reinterpret_cast<uint32_t*>(smem);
-  uint32_t* wpre = mask + mask_words_padded(G.Bd);
-  uint32_t* W = wpre + mask_words_padded(G.Bd);  // 16-byte aligned
-  uint32_t* nxt = W + E;
-  uint32_t* head = nxt + E;
-  uint32_t* queue = head + Ucap;   // union ranks found in several rows
-  uint32_t* scan = queue + Ucap;
-  uint32_t* qcount = scan + T / 32;
+  uint16_t* wpre = reinterpret_cast<uint16_t*>(mask + WnP);
+  uint32_t* W = reinterpret_cast<uint32_t*>(wpre + ((WnP + 7) & ~7));  // 16-byte aligned
+  float2* acc = reinterpret_cast<float2*>(W + E);
+  uint16_t* uidx = reinterpret_cast<uint16_t*>(acc + Ucap);
+  uint32_t* scan = reinterpret_cast<uint32_t*>(uidx + Ucap);
 
   for (int w = tid; w < Wn; w += T) mask[w] = 0u;
-  for (int u = tid; u < Ucap; u += T) head[u] = kNil;
-  if (tid == 0) *qcount = 0u;
   __syncthreads();
 
   // Rows of steps t, t-1, ..., t-rows+1 (age 0 = this step's row), staged 4
@@ -428,20 +430,26 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   }
   __syncthreads();
 
+  // Union rank of each mask word (T >= Wn: one word per thread).
   const uint32_t pc = (tid < Wn) ? (uint32_t)__popc(mask[tid]) : 0u;
   uint32_t U;
   const uint32_t incl = block_scan_1bar<T, uint32_t>(pc, scan, U);
-  if (tid < Wn) wpre[tid] = incl - pc;
+  if (tid < Wn) wpre[tid] = (uint16_t)(incl - pc);
   __syncthreads();
 
+  // Each staged entry: index -> union rank (U <= 15360, so a rank never equals
+  // the empty marker 0xFFFF); every slot's accumulator is cleared and its
+  // index recorded (entries of one index write the same values).
   const int staged = A.rows * G.kp;
   for (int e = tid; e < staged; e += T) {
-    const uint32_t idx = W[e] & 0xFFFFu;
+    const uint32_t v = W[e];
+    const uint32_t idx = v & 0xFFFFu;
     if (idx >= (uint32_t)L) continue;
     const uint32_t w = idx >> 5;
     const uint32_t rank = wpre[w] + (uint32_t)__popc(mask[w] & ((1u << (idx & 31)) - 1u));
-    const uint32_t age = __umulhi((uint32_t)e, A.kp_recip);
-    nxt[e] = atomicExch(&head[rank], (age << 16) | (uint32_t)e);
+    W[e] = (v & 0xFFFF0000u) | rank;
+    uidx[rank] = (uint16_t)idx;
+    acc[rank] = make_float2(0.0f, 0.0f);
   }
   if (A.has_decay) {
     float* pb = A.params + start;
@@ -449,12 +457,27 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   }
   __syncthreads();
 
-  // Pass 1, uniform across lanes: indices present in one row only (the common
-  // case); the others are queued. Up to kBatch indices per thread per round,
-  // all parameter loads issued before any store so the read-modify-writes
-  // overlap in flight. u = m_hat / (eps + sqrt(v_hat)) uses the hardware
-  // square root and reciprocal approximations (a few ulp, far inside the fp32
-  // update's error).
+  // The sums, one row at a time from the oldest: z <- z + beta^age * V.
+  for (int age = A.rows - 1; age >= 0; --age) {
+    const float c1 = s_w1[age], c2 = s_w2[age];
+    const uint32_t* Wr = W + age * G.kp;
+    for (int p = tid; p < G.kp; p += T) {
+      const uint32_t v = Wr[p];
+      const uint32_t r = v & 0xFFFFu;
+      if (r == 0xFFFFu) continue;
+      const float V = __uint_as_float(v & 0xFFFF0000u);
+      float2 z = acc[r];
+      z.x = __fadd_rn(z.x, __fmul_rn(c1, V));
+      z.y = __fadd_rn(z.y, __fmul_rn(c2, __fmul_rn(V, V)));
+      acc[r] = z;
+    }
+    __syncthreads();
+  }
+
+  // Parameter update on the union, up to kBatch slots per thread per round
+  // with all parameter loads issued before any store. u = m_hat/(eps+sqrt(v_hat))
+  // uses the hardware square root and reciprocal approximations (a few ulp,
+  // far inside the fp32 update's error).
   constexpr int kBatch = 4;
   for (uint32_t r0 = 0; r0 < U; r0 += kBatch * T) {
     uint32_t idx[kBatch];
@@ -465,17 +488,10 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
       idx[b] = kNil;
       mh[b] = vh[b] = pv[b] = 0.0f;
       if (r >= U) continue;
-      const uint32_t h = head[r];
-      if (nxt[h & 0xFFFFu] != kNil) {
-        queue[atomicAdd(qcount, 1u)] = r;
-        continue;
-      }
-      const uint32_t bv = W[h & 0xFFFFu];
-      const int age = (int)(h >> 16);
-      const float V = __uint_as_float(bv & 0xFFFF0000u);
-      idx[b] = bv & 0xFFFFu;
-      mh[b] = __fmul_rn(A.f1, __fmul_rn(s_w1[age], V));
-      vh[b] = __fmul_rn(A.f2, __fmul_rn(s_w2[age], __fmul_rn(V, V)));
+      idx[b] = uidx[r];
+      const float2 z = acc[r];
+      mh[b] = __fmul_rn(A.f1, z.x);
+      vh[b] = __fmul_rn(A.f2, z.y);
       pv[b] = A.params[start + idx[b]];
     }
 #pragma unroll
@@ -487,41 +503,6 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
         A.mhat[start + idx[b]] = mh[b];
         A.vhat[start + idx[b]] = vh[b];
       }
-    }
-  }
-  __syncthreads();
-
-  // Pass 2: indices present in several rows, summed oldest row first.
-  const uint32_t nq = *qcount;
-  for (uint32_t qi = tid; qi < nq; qi += T) {
-    const uint32_t h = head[queue[qi]];
-    const uint32_t idx = W[h & 0xFFFFu] & 0xFFFFu;
-    float z1 = 0.0f, z2 = 0.0f;
-    int prev = 1 << 30;
-    for (;;) {
-      int best = -1;
-      uint32_t bv = 0u;
-      for (uint32_t l = h; l != kNil; l = nxt[l & 0xFFFFu]) {
-        const int age = (int)(l >> 16);
-        if (age < prev && age > best) {
-          best = age;
-          bv = W[l & 0xFFFFu];
-        }
-      }
-      if (best < 0) break;
-      const float V = __uint_as_float(bv & 0xFFFF0000u);
-      z1 = __fadd_rn(z1, __fmul_rn(s_w1[best], V));
-      z2 = __fadd_rn(z2, __fmul_rn(s_w2[best], __fmul_rn(V, V)));
-      prev = best;
-    }
-    const float mh = __fmul_rn(A.f1, z1);
-    const float vh = __fmul_rn(A.f2, z2);
-    const float u = __fmul_rn(mh, rcp_approx(__fadd_rn(A.eps, sqrt_approx(vh))));
-    float* pp = A.params + start + idx;
-    *pp = __fsub_rn(*pp, __fmul_rn(A.lr, u));
-    if (A.mhat) {
-      A.mhat[start + idx] = mh;
-      A.vhat[start + idx] = vh;
     }
   }
 }

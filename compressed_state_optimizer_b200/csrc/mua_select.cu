@@ -507,7 +507,7 @@ __device__ __forceinline__ void select_block(const StepArgs& A, int j,
 template <int T, bool VEC>
 __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
     mua_select_kernel(const StepArgs A) {
-  extern __shared__ __align__(16) uint8_t dyn[];
+  extern __shared__ __align__(128) uint8_t dyn[];
   __shared__ SelectShared sh;
   const int j = blockIdx.x;
   const int64_t start = (int64_t)j * A.g.Bd;

@@ -73,7 +73,8 @@ typedef struct mua_ctx* mua_t;
  *   out          receives the handle (release with mua_destroy)
  * Errors: MUA_ERR_ARG for out-of-range values or NULL out;
  * MUA_ERR_UNSUPPORTED when bits != 4 or when the window of one block,
- * m * k_b entries, is too large for the on-chip AdamStats (more than 16384).
+ * m * k_b entries, is too large for the on-chip AdamStats (m * k_b rounded up
+ * to a multiple of 4 per row, more than 15360 entries).
  */
 int mua_create(int64_t d, int32_t block_size, int32_t k_per_block, int32_t window,
                int32_t bits, mua_t* out);

@@ -65,6 +65,7 @@ def _create(mua, *args):
     ((100, 16384, 164, 65, 4), -1),        # m > 64
     ((100, 16384, 164, 10, 8), -2),        # b != 4
     ((100, 16384, 16384, 10, 4), -2),      # window of a block too large for the chip
+    ((100, 16384, 1537, 10, 4), -2),       # m * kp = 15400 > 15360
 ])
 def test_create_rejects(mua, args, code):
     rc, h = _create(mua, *args)
@@ -73,7 +74,8 @@ def test_create_rejects(mua, args, code):
 
 
 def test_create_accepts_limits(mua):
-    for args in [(1, 2, 1, 1, 4), (32766 * 3 + 5, 32766, 328, 10, 4), (10**12, 16384, 164, 64, 4)]:
+    for args in [(1, 2, 1, 1, 4), (32766 * 3 + 5, 32766, 328, 10, 4), (10**12, 16384, 164, 64, 4),
+                 (100, 32766, 1536, 10, 4)]:
         rc, h = _create(mua, *args)
         assert rc == 0 and h.value
         mua.library().mua_destroy(h)
