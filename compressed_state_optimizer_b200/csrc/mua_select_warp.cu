@@ -12,16 +12,20 @@
 // blocks are in flight per SM and memory latency hides behind the others.
 //
 // Exact Top-k:
-//  * candidate path (blocks of at least 4096 entries): 512 sample keys (64
-//    16-byte chunks spread over the block), each lane's top-2, a warp sort of
-//    those 64 values -> tau_lo (aiming at ~2.5k candidates); one streaming pass
-//    writes every |a| >= tau_lo to the warp's list in index order and folds
-//    the rest into the residual min/max; an exact warp radix select on the
-//    list (8-bit digits from the highest bit where tau_lo and the list maximum
-//    differ) finds the k-th key, and one warp scan places the entries;
-//  * fallback (small blocks, or fewer than k / more than kWarpCap candidates):
-//    exact radix select on all keys by streaming passes over the block (it is
-//    in L2 by then), 8 bits per pass, then one placing pass.
+//  * candidate path (blocks of 4096 to 16384 entries): 512 sample keys (64
+//    chunks of 8 spread over the block), each lane's top-2, a warp sort of
+//    those 64 values -> tau_lo (aiming at ~2.5k candidates); one streaming
+//    pass (lane l holds elements 256 s + 8 l .. + 7 of step s) appends every
+//    |a| >= tau_lo to the lane's own strided region of the list, with no
+//    cross-lane step, and folds the rest into the residual min/max; an exact
+//    warp radix select on the list (8-bit digits from the highest bit where
+//    tau_lo and the list maximum differ) finds the k-th key; the selected
+//    entries are marked in a bitmask of the block (ties at the threshold by a
+//    lowest-index merge of the lanes' regions, each already in index order)
+//    and a popcount prefix of the mask gives each its place in the row;
+//  * fallback (small blocks, or fewer than k / more than kLaneCap candidates
+//    in a lane): exact radix select on all keys by streaming passes over the
+//    block (it is in L2 by then), 8 bits per pass, then one placing pass.
 // HBM traffic per parameter: 2 B gradient + 0.5 B codes read; per selected
 // entry 4 B written.
 #include "mua_kernels.cuh"
@@ -31,12 +35,15 @@ namespace {
 
 constexpr int kWarps = 8;         // warps (= blocks in flight) per CTA
 constexpr int kWarpCap = 1024;    // candidate list entries per warp
+constexpr int kLaneCap = kWarpCap / 32;  // entries per lane region
+constexpr int kSelMaskWords = 512;       // selection bitmask: blocks of up to 16384
 constexpr int kUnroll = 4;        // 256-element steps loaded ahead
 
 struct WarpSmem {
-  uint32_t bits[kWarpCap];
-  uint16_t idx[kWarpCap];
-  uint32_t hist[256];
+  uint32_t bits[kWarpCap];  // a_t bits; lane l's i-th candidate at [32 i + l]
+  uint16_t idx[kWarpCap];   // its block-relative index
+  uint32_t hist[256];       // radix histogram, then the mask's u16 word prefix
+  uint32_t mask[kSelMaskWords];
 };
 
 struct CtaSmem {
@@ -86,6 +93,55 @@ __device__ __forceinline__ void dequant8(const uint4& gv, uint32_t cv, const flo
     const float a = __fadd_rn(__uint_as_float(grad_bits(gv, e)), lv[(cv >> (4 * e)) & 0xFu]);
     ab[e] = (e0 + e < L) ? __float_as_uint(a) : 0u;
   }
+}
+
+// dequant8 for a step wholly inside the block. The code word is pre-scaled by 4
+// so each nibble becomes a byte offset into the level table directly.
+__device__ __forceinline__ void dequant8_full(const uint4& gv, uint32_t cv, const float* lv,
+                                              uint32_t (&ab)[kChunk]) {
+  const uint32_t c4 = cv << 2;
+  const char* lb = reinterpret_cast<const char*>(lv);
+#pragma unroll
+  for (int e = 0; e < kChunk; ++e) {
+    const uint32_t off = (e == 0) ? (c4 & 0x3Cu) : ((cv >> (4 * e - 2)) & 0x3Cu);
+    const float a = __fadd_rn(__uint_as_float(grad_bits(gv, e)),
+                              *reinterpret_cast<const float*>(lb + off));
+    ab[e] = __float_as_uint(a);
+  }
+}
+
+// Per-lane state of the candidate pass.
+struct LaneState {
+  uint32_t cnt;  // entries in the lane's region
+  uint32_t tau;  // candidate threshold of the lane (>= the warp's tau_lo)
+  float rmin, rmax;
+};
+
+// Makes room in a lane's region for one more 8-element step: while it holds
+// more than kLaneCap - 8 entries, the smallest is dropped into the residual's
+// min/max (its slot takes the region's last entry) and the lane's threshold
+// rises above it, so every key the lane ever drops is below its final tau.
+__device__ __forceinline__ LaneState make_room(uint32_t* bits, uint16_t* idx, int lane,
+                                            LaneState st) {
+  while (st.cnt > (uint32_t)(kLaneCap - kChunk)) {
+    uint32_t m0 = 0xFFFFFFFFu, at = 0u;
+    for (uint32_t i = 0; i < st.cnt; ++i) {
+      const uint32_t key = bits[32 * i + lane] & 0x7FFFFFFFu;
+      if (key < m0) {
+        m0 = key;
+        at = i;
+      }
+    }
+    const float v = __uint_as_float(bits[32 * at + lane]);
+    st.rmin = fminf(st.rmin, v);
+    st.rmax = fmaxf(st.rmax, v);
+    st.tau = max(st.tau, m0 + 1u);
+    const uint32_t last = st.cnt - 1u;
+    bits[32 * at + lane] = bits[32 * last + lane];
+    idx[32 * at + lane] = idx[32 * last + lane];
+    st.cnt = last;
+  }
+  return st;
 }
 
 __device__ __forceinline__ void put_row(uint32_t* row, uint32_t pos, int k, uint32_t idx,
@@ -171,7 +227,7 @@ __device__ __forceinline__ void warp_radix(int hi, uint32_t prefix, int k, uint3
 }
 
 template <bool VEC>
-__global__ void __launch_bounds__(kWarps * 32) mua_select_warp_kernel(const StepArgs A) {
+__global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const StepArgs A) {
   extern __shared__ __align__(16) uint8_t dyn[];
   CtaSmem& S = *reinterpret_cast<CtaSmem*>(dyn);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -196,7 +252,7 @@ __global__ void __launch_bounds__(kWarps * 32) mua_select_warp_kernel(const Step
   bool done = false;
 
   // ---------------- candidate path
-  if (L >= 4096 && 8 * k <= L) {
+  if (L >= 4096 && L <= 32 * kSelMaskWords && 8 * k <= L) {
     // 512 samples: 64 chunks of 8, chunk c at element (c * (L / 64)) & ~7.
     const int cstride = (L / 64) & ~7;
     uint32_t t1 = 0u, t2 = 0u;  // this lane's two largest sample keys
@@ -243,95 +299,142 @@ __global__ void __launch_bounds__(kWarps * 32) mua_select_warp_kernel(const Step
     const int r = min(63, (5 * k + 63) / 64 - 1);  // ~2.5k of 32x as many elements
     const uint32_t tl0 = __shfl_sync(0xFFFFFFFFu, v0, r >> 1);
     const uint32_t tl1 = __shfl_sync(0xFFFFFFFFu, v1, r >> 1);
-    const uint32_t tau_lo = (r & 1) ? tl1 : tl0;
+    const uint32_t tau_first = (r & 1) ? tl1 : tl0;
+    const uint32_t tau_retry = __shfl_sync(0xFFFFFFFFu, v1, 31);  // smallest of the 64
 
-    // One streaming pass: candidates to the list in index order.
-    uint32_t n = 0u;  // list length so far (warp-uniform)
-    uint32_t kmax = 0u;
-    for (int s0 = 0; s0 < nsteps; s0 += kUnroll) {
-      uint4 gv[kUnroll];
-      uint32_t cv[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int e0 = ((s0 + u) << 8) + 8 * lane;
-        if (s0 + u < nsteps) load_step<VEC>(A.grads, A.codes, start, L, e0, gv[u], cv[u]);
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        if (s0 + u >= nsteps) break;
-        const int e0 = ((s0 + u) << 8) + 8 * lane;
-        uint32_t ab[kChunk];
-        dequant8(gv[u], cv[u], lv, e0, L, ab);
-        uint32_t cnt = 0u;
-#pragma unroll
-        for (int e = 0; e < kChunk; ++e) {
-          const uint32_t key = ab[e] & 0x7FFFFFFFu;
-          const bool cand = key >= tau_lo && e0 + e < L;
-          cnt += cand;
-          const float v = cand ? 0.0f : __uint_as_float(ab[e]);
-          rmin = fminf(rmin, v);
-          rmax = fmaxf(rmax, v);
+    // One streaming pass per attempt (a second, with a lower tau_lo, only when
+    // the first finds fewer than k candidates).
+    for (int attempt = 0; attempt < 2 && !done; ++attempt) {
+      const uint32_t tau_lo = attempt == 0 ? tau_first : tau_retry;
+      if (attempt == 1 && tau_retry >= tau_first) break;
+      // Candidates (key >= tau) go to the lane's region. Before each step a
+      // lane with fewer than 8 free slots drops its smallest entries and
+      // raises its tau (make_room), so a step's appends always fit. The
+      // result is exact when every raised tau is at most the final
+      // threshold (checked below).
+      LaneState ls{0u, tau_lo, 0.0f, 0.0f};
+      auto scan_step = [&](const uint32_t (&ab)[kChunk], int e0, bool full) {
+        if (__any_sync(0xFFFFFFFFu, ls.cnt > (uint32_t)(kLaneCap - kChunk))) {
+          if (ls.cnt > (uint32_t)(kLaneCap - kChunk)) ls = make_room(W.bits, W.idx, lane, ls);
+          __syncwarp();
         }
-        const uint32_t incl = warp_incl_scan(cnt, lane);
-        uint32_t pos = n + incl - cnt;
-        n += __shfl_sync(0xFFFFFFFFu, incl, 31);
 #pragma unroll
         for (int e = 0; e < kChunk; ++e) {
           const uint32_t key = ab[e] & 0x7FFFFFFFu;
-          if (key >= tau_lo && e0 + e < L) {
-            if (pos < (uint32_t)kWarpCap) {
-              W.bits[pos] = ab[e];
-              W.idx[pos] = (uint16_t)(e0 + e);
-            }
-            kmax = max(kmax, key);
-            ++pos;
+          const bool cand = key >= ls.tau && (full || e0 + e < L);
+          if (cand) {
+            W.bits[(ls.cnt << 5) | (uint32_t)lane] = ab[e];
+            W.idx[(ls.cnt << 5) | (uint32_t)lane] = (uint16_t)(e0 + e);
           }
+          ls.cnt += cand ? 1u : 0u;
+          const float v = cand ? 0.0f : __uint_as_float(ab[e]);
+          ls.rmin = fminf(ls.rmin, v);
+          ls.rmax = fmaxf(ls.rmax, v);
+        }
+      };
+      const int nfull = L >> 8;  // steps with all 256 elements inside the block
+      for (int s0 = 0; s0 < nfull; s0 += kUnroll) {
+        uint4 gv[kUnroll];
+        uint32_t cv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int e0 = ((s0 + u) << 8) + 8 * lane;
+          if (s0 + u < nfull) load_step<VEC>(A.grads, A.codes, start, L, e0, gv[u], cv[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          if (s0 + u >= nfull) break;
+          uint32_t ab[kChunk];
+          dequant8_full(gv[u], cv[u], lv, ab);
+          scan_step(ab, ((s0 + u) << 8) + 8 * lane, true);
         }
       }
-    }
-    __syncwarp();
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
-    if (n >= (uint32_t)k && n <= (uint32_t)kWarpCap) {
-      if (lane == 0 && kmax >= 0x7F800000u) atomicOr(&A.hdr[kHdrStatus], kStatusNonFinite);
-      const int q = ((int)n + 31) >> 5;
-      const int i0 = min((int)n, lane * q), i1 = min((int)n, i0 + q);
+      if (nfull < nsteps) {  // the block's partial last step
+        const int e0 = (nfull << 8) + 8 * lane;
+        uint4 gv;
+        uint32_t cv;
+        load_step<VEC>(A.grads, A.codes, start, L, e0, gv, cv);
+        uint32_t ab[kChunk];
+        dequant8(gv, cv, lv, e0, L, ab);
+        scan_step(ab, e0, false);
+      }
+      rmin = ls.rmin;
+      rmax = ls.rmax;
+      const uint32_t cnt = ls.cnt;
+      const int mine = (int)cnt;
+      const uint32_t n = __reduce_add_sync(0xFFFFFFFFu, cnt);
+      const uint32_t drop_bound = __reduce_max_sync(0xFFFFFFFFu, ls.tau > tau_lo ? ls.tau : 0u);
+      __syncwarp();
+      if (n < (uint32_t)k) continue;  // too few: retry lower, else the fallback
+      uint32_t kmax = 0u;
+      for (int i = 0; i < mine; ++i) kmax = max(kmax, W.bits[32 * i + lane] & 0x7FFFFFFFu);
+      kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
       int mode = 1, need = k;
       uint32_t thr = tau_lo;
       const uint32_t diff = kmax ^ tau_lo;
       if (diff != 0u) {
         warp_radix(31 - __clz(diff), tau_lo, k, W.hist, lane,
                    [&](auto&& f) {
-                     for (int i = i0; i < i1; ++i) f(W.bits[i] & 0x7FFFFFFFu);
+                     for (int i = 0; i < mine; ++i) f(W.bits[32 * i + lane] & 0x7FFFFFFFu);
                    },
                    mode, thr, need);
       }
-      // positions in index order over the list
-      uint32_t cg = 0u, ce = 0u;
-      for (int i = i0; i < i1; ++i) {
-        const uint32_t key = W.bits[i] & 0x7FFFFFFFu;
-        if (mode == 0) {
-          cg += key >= thr;
-        } else {
-          cg += key > thr;
-          ce += key == thr;
+      // Exact only if every dropped key (< its lane's tau <= drop_bound) is below thr.
+      if (drop_bound > thr) break;
+      if (lane == 0 && kmax >= 0x7F800000u) atomicOr(&A.hdr[kHdrStatus], kStatusNonFinite);
+      // Selection bitmask: keys above the threshold (at or above it in mode 0) ...
+      const int wn = (L + 31) >> 5;
+      for (int w = lane; w < wn; w += 32) W.mask[w] = 0u;
+      __syncwarp();
+      for (int i = 0; i < mine; ++i) {
+        const uint32_t key = W.bits[32 * i + lane] & 0x7FFFFFFFu;
+        if (mode == 0 ? key >= thr : key > thr) {
+          const uint32_t idx = W.idx[32 * i + lane];
+          atomicOr(&W.mask[idx >> 5], 1u << (idx & 31));
         }
       }
-      const uint32_t packed = cg | (ce << 16);
-      const uint32_t x = warp_incl_scan(packed, lane) - packed;
-      uint32_t run_g = x & 0xFFFFu, run_e = x >> 16;
-      for (int i = i0; i < i1; ++i) {
-        const uint32_t bits = W.bits[i];
-        const uint32_t key = bits & 0x7FFFFFFFu;
-        const bool gt = (mode == 0) ? key >= thr : key > thr;
-        if (gt) {
-          put_row(row, run_g + min(run_e, (uint32_t)need), k, W.idx[i], bits);
-          ++run_g;
-        } else if (mode == 1 && key == thr && run_e < (uint32_t)need) {
-          put_row(row, run_g + run_e, k, W.idx[i], bits);
-          ++run_e;
+      // ... and, in mode 1, the `need` lowest indices among keys equal to it,
+      // one per round: the lowest unmarked tied index over all lanes.
+      if (mode == 1) {
+        for (int q = 0; q < need; ++q) {
+          __syncwarp();
+          uint32_t head = 0xFFFFu;
+          for (int i = 0; i < mine; ++i) {
+            if ((W.bits[32 * i + lane] & 0x7FFFFFFFu) != thr) continue;
+            const uint32_t idx = W.idx[32 * i + lane];
+            if (idx < head && !((W.mask[idx >> 5] >> (idx & 31)) & 1u)) head = idx;
+          }
+          const uint32_t low = __reduce_min_sync(0xFFFFFFFFu, head);
+          if (head == low && head != 0xFFFFu) atomicOr(&W.mask[head >> 5], 1u << (head & 31));
+        }
+      }
+      __syncwarp();
+      // u16 exclusive popcount prefix of the mask words (lane l: words 16 l ..)
+      uint16_t* wpre = reinterpret_cast<uint16_t*>(W.hist);
+      {
+        const int w0 = 16 * lane;
+        uint32_t c = 0u;
+#pragma unroll
+        for (int w = 0; w < 16; ++w) c += (w0 + w < wn) ? (uint32_t)__popc(W.mask[w0 + w]) : 0u;
+        uint32_t run = warp_incl_scan(c, lane) - c;
+#pragma unroll
+        for (int w = 0; w < 16; ++w) {
+          if (w0 + w < wn) {
+            wpre[w0 + w] = (uint16_t)run;
+            run += (uint32_t)__popc(W.mask[w0 + w]);
+          }
+        }
+      }
+      __syncwarp();
+      // Place the selected entries; the others join the residual's min/max.
+      for (int i = 0; i < mine; ++i) {
+        const uint32_t bits = W.bits[32 * i + lane];
+        const uint32_t idx = W.idx[32 * i + lane];
+        const uint32_t word = W.mask[idx >> 5];
+        if ((word >> (idx & 31)) & 1u) {
+          const uint32_t pos = wpre[idx >> 5] + (uint32_t)__popc(word & ((1u << (idx & 31)) - 1u));
+          put_row(row, pos, k, idx, bits);
         } else {
-          if (mode == 1 && key == thr) ++run_e;
           rmin = fminf(rmin, __uint_as_float(bits));
           rmax = fmaxf(rmax, __uint_as_float(bits));
         }

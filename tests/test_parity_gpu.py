@@ -201,3 +201,39 @@ def test_deterministic_and_resumable():
     saved_s, saved_p = s3.cpu().clone(), p3.cpu().clone()
     s4, p4 = run(5, saved_s.cuda(), saved_p.cuda(), t0=6)
     assert torch.equal(s4, s1) and torch.equal(p4, p1)
+
+
+def _structured_grads(d, Bd, seed):
+    """Blocks built to drive the select kernel through each of its paths.
+
+    Block j % 4 == 0: the large values sit only on the 512 elements the
+    threshold sample reads (64 runs of 8 at stride 256), so the first
+    candidate pass finds too few entries; 1: all large values on one
+    lane's elements (elements 40..47 of every 256), so that lane holds the
+    whole Top-k; 2: plain; 3: one lane's elements 30 % larger than the rest
+    (that lane's region tends to fill). The oracle decides what is right."""
+    import torch
+
+    def fn(t):
+        rng = np.random.default_rng(seed + t)
+        g = (rng.standard_normal(d) * 0.01).astype(np.float32)
+        steps = np.arange(64)[:, None] * 256
+        for j in range(d // Bd):
+            base = j * Bd
+            if j % 4 == 0:
+                pos = (steps + np.arange(8)).ravel()
+                g[base + pos] = rng.standard_normal(pos.size)
+            elif j % 4 == 1:
+                pos = (steps + 40 + np.arange(8)).ravel()
+                g[base + pos] = rng.standard_normal(pos.size)
+            elif j % 4 == 3:
+                pos = (steps + 24 + np.arange(8)).ravel()
+                g[base + pos] *= 1.3
+        return torch.from_numpy(g).to(torch.bfloat16)
+    return fn
+
+
+@pytest.mark.parametrize("kb", [164, 600])
+def test_select_paths(kb):
+    d, Bd = 8 * 16384 + 999, 16384
+    run_parity(d, Bd, kb, 3, 4, grads_fn=_structured_grads(d, Bd, 99 + kb))
