@@ -10,7 +10,7 @@
 //   and, for the blocks the select kernel left (j & 7 >= update_split), the
 //   AdamStats update of the block's parameters (block_update).
 // Blocks run in reverse order, so the first blocks find the tail of the
-// select kernel's reads still in L2. HBM traffic per parameter: 2.5 B read
+// select kernel's reads in L2. HBM traffic per parameter: 2.5 B read
 // (g, e) + 0.5 B written (e); plus block_update's traffic for its blocks.
 #include "mua_kernels.cuh"
 
@@ -19,17 +19,20 @@ namespace {
 
 template <int T, bool VEC>
 __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
-    mua_apply_kernel(const StepArgs A) {
+    mua_apply_kernel(const __grid_constant__ StepArgs A) {
   extern __shared__ __align__(16) uint8_t dyn[];
   __shared__ float s_lv[16];
   __shared__ float s_w1[kMaxWindow], s_w2[kMaxWindow];
-  uint32_t* sel = reinterpret_cast<uint32_t*>(dyn);  // [Wn] bits of the new row
 
   const int tid = threadIdx.x;
   const Geometry& G = A.g;
   const int j = G.nb - 1 - (int)blockIdx.x;
   const int64_t start = (int64_t)j * G.Bd;
   const int L = (j == G.nb - 1) ? G.last_len : G.Bd;
+
+  load_weights(A, s_w1, s_w2);
+
+  uint32_t* sel = reinterpret_cast<uint32_t*>(dyn);  // [Wn] bits of the new row
   const int Wn = (G.Bd + 31) >> 5;
 
   // Issue the streaming loads first; they land while the new row is read.
@@ -40,7 +43,6 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
   const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
   const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
   fill_levels(s_lv, delta, __fdiv_rn(__fsub_rn(Delta, delta), 15.0f));
-  load_weights(A, s_w1, s_w2);
   for (int w = tid; w < Wn; w += T) sel[w] = 0u;
   __syncthreads();
   {
@@ -58,6 +60,7 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
   const float inv16 =
       (Dn == dn) ? 0.0f : __fmul_rn(__fdiv_rn(15.0f, __fsub_rn(Dn, dn)), 65536.0f);
   const uint64_t grp0 = (uint64_t)(G.base_index + start) >> 3;  // VEC: start % 8 == 0
+  const char* lvb = reinterpret_cast<const char*>(s_lv);
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
     const int e0 = elem_index<T>(c, tid, 0);
@@ -70,7 +73,9 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
 #pragma unroll
       for (int e = 0; e < kChunk; ++e) {
         const float gf = __uint_as_float(grad_bits(gv[c], e));
-        float a = __fadd_rn(gf, s_lv[(cv[c] >> (4 * e)) & 0xFu]);
+        // the code nibble as a byte offset into the level table
+        const uint32_t off = (e == 0) ? ((cv[c] << 2) & 0x3Cu) : ((cv[c] >> (4 * e - 2)) & 0x3Cu);
+        float a = __fadd_rn(gf, *reinterpret_cast<const float*>(lvb + off));
         if ((selbits >> e) & 1u) a = 0.0f;
         const float s16 = __fmul_rn(__fsub_rn(a, dn), inv16);
         const uint32_t xw = chunk_word(x, e >> 1);
@@ -107,9 +112,7 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
       for (int e = 0; e < nval; e += 2) cdst[e >> 1] = (uint8_t)(pack >> (4 * e));
     }
   }
-
-  // (6) for the blocks the select kernel left.
-  if (!update_in_select(A, j)) {
+  if (!update_in_select(A, j)) {  // (6) AdamStats update of block j
     __syncthreads();
     block_update<T>(A, j, start, L, dyn, s_w1, s_w2);
   }

@@ -172,7 +172,7 @@ __device__ __forceinline__ void dequant_block(const uint4 (&gv)[kChunks],
 // result (bits 0..15 are scratch); the caller shifts it into place.
 __device__ __forceinline__ uint32_t quantize_code_hi(float s16, uint32_t r) {
   const uint32_t big = __float_as_uint(__fadd_rz(s16, 8388608.0f));  // 0x4B000000 + floor
-  return min(big + r, 0x4B0FFFFFu);
+  return __viaddmin_u32(big, r, 0x4B0FFFFFu);  // min(big + r, code 15)
 }
 
 // ---------------------------------------------------------------- TMA bulk copies
@@ -507,15 +507,13 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   }
 }
 
-// Copies the AdamStats weights into shared memory with constant indices (so
-// they stay in the kernel's parameter bank). Caller synchronizes.
+// Copies the AdamStats weights into shared memory, one per thread (A must be
+// the kernel's __grid_constant__ argument, so the indexed reads stay in the
+// parameter bank). Caller synchronizes.
 __device__ __forceinline__ void load_weights(const StepArgs& A, float* s_w1, float* s_w2) {
-  if (threadIdx.x == 0) {
-#pragma unroll
-    for (int r = 0; r < kMaxWindow; ++r) {
-      s_w1[r] = A.w1[r];
-      s_w2[r] = A.w2[r];
-    }
+  for (int r = threadIdx.x; r < kMaxWindow; r += blockDim.x) {
+    s_w1[r] = A.w1[r];
+    s_w2[r] = A.w2[r];
   }
 }
 

@@ -506,7 +506,7 @@ __device__ __forceinline__ void select_block(const StepArgs& A, int j,
 // One CTA per block.
 template <int T, bool VEC>
 __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
-    mua_select_kernel(const StepArgs A) {
+    mua_select_kernel(const __grid_constant__ StepArgs A) {
   extern __shared__ __align__(128) uint8_t dyn[];
   __shared__ SelectShared sh;
   const int j = blockIdx.x;
@@ -533,7 +533,7 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
 // Shared memory: stage {bf16 g[B_d], codes[B_d/2]}, then `work`.
 template <int T>
 __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
-    mua_select_persistent(const StepArgs A) {
+    mua_select_persistent(const __grid_constant__ StepArgs A) {
   extern __shared__ __align__(128) uint8_t dyn[];
   __shared__ SelectShared sh;
   __shared__ __align__(8) uint64_t bar;
