@@ -70,18 +70,26 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
     if (VEC) {
       const uint64_t grp = grp0 + (uint64_t)(c * T + tid);
       const uint4 x = philox4x32_10((uint32_t)grp, (uint32_t)(grp >> 32), A.t_lo, A.t_hi, A.keys);
+      const uint64_t dn2 = f2_pack(dn, dn), inv2 = f2_pack(inv16, inv16);
+      const uint64_t magic2 = f2_pack(8388608.0f, 8388608.0f);
 #pragma unroll
-      for (int e = 0; e < kChunk; ++e) {
-        const float gf = __uint_as_float(grad_bits(gv[c], e));
-        // the code nibble as a byte offset into the level table
-        const uint32_t off = (e == 0) ? ((cv[c] << 2) & 0x3Cu) : ((cv[c] >> (4 * e - 2)) & 0x3Cu);
-        float a = __fadd_rn(gf, *reinterpret_cast<const float*>(lvb + off));
-        if ((selbits >> e) & 1u) a = 0.0f;
-        const float s16 = __fmul_rn(__fsub_rn(a, dn), inv16);
+      for (int e = 0; e < kChunk; e += 2) {  // elements e, e + 1: gradient word e / 2
+        const uint32_t w = chunk_word(gv[c], e >> 1);
+        const uint32_t off0 = (e == 0) ? ((cv[c] << 2) & 0x3Cu) : ((cv[c] >> (4 * e - 2)) & 0x3Cu);
+        const uint32_t off1 = (cv[c] >> (4 * e + 2)) & 0x3Cu;
+        const uint64_t g2 = ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint32_t)(w << 16);
+        const uint64_t l2 = f2_pack(*reinterpret_cast<const float*>(lvb + off0),
+                                    *reinterpret_cast<const float*>(lvb + off1));
+        uint64_t a2 = f2_add_rn(g2, l2);
+        if ((selbits >> e) & 1u) a2 &= 0xFFFFFFFF00000000ull;  // selected: a = +0
+        if ((selbits >> (e + 1)) & 1u) a2 &= 0x00000000FFFFFFFFull;
+        const uint64_t big2 = f2_add_rz(f2_mul_rn(f2_sub_rn(a2, dn2), inv2), magic2);
         const uint32_t xw = chunk_word(x, e >> 1);
-        const uint32_t r = (e & 1) ? (xw >> 16) : (xw & 0xFFFFu);
-        const uint32_t hi = quantize_code_hi(s16, r);
-        pack |= (e <= 4 ? (hi >> (16 - 4 * e)) : (hi << (4 * e - 16))) & (0xFu << (4 * e));
+        // floor(s16) sits in the low mantissa of 2^23 + s16 (rounded toward zero)
+        const uint32_t hi0 = __viaddmin_u32((uint32_t)big2, xw & 0xFFFFu, 0x4B0FFFFFu);
+        const uint32_t hi1 = __viaddmin_u32((uint32_t)(big2 >> 32), xw >> 16, 0x4B0FFFFFu);
+        pack |= (e <= 4 ? (hi0 >> (16 - 4 * e)) : (hi0 << (4 * e - 16))) & (0xFu << (4 * e));
+        pack |= (e + 1 <= 4 ? (hi1 >> (12 - 4 * e)) : (hi1 << (4 * e - 12))) & (0xFu << (4 * e + 4));
       }
     } else {
       const int64_t gidx = G.base_index + start + e0;

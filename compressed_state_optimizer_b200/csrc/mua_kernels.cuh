@@ -141,6 +141,35 @@ __device__ __forceinline__ uint32_t grad_bits(const uint4& v, int e) {
   return (e & 1) ? (word & 0xFFFF0000u) : (word << 16);
 }
 
+// Two-wide fp32 arithmetic (sm_100 packed f32x2 instructions): each half is
+// the IEEE operation with the stated rounding, bit for bit the scalar result;
+// one instruction issues both. A pair is (low = x, high = y).
+__device__ __forceinline__ uint64_t f2_pack(float x, float y) {
+  return ((uint64_t)__float_as_uint(y) << 32) | __float_as_uint(x);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_add_rn(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add_rz(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub_rn(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_mul_rn(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // Q^{-1} levels delta + c * unit for c = 0..15, each computed as
 // fl(delta + fl(fl(c) * unit)) exactly as [MicroAdam ¶1]'s dequantization is
 // written; threads 0..15 fill the table, the caller synchronizes.
