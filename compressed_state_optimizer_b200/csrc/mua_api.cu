@@ -28,7 +28,8 @@ struct mua_ctx {
   int64_t nb;           // blocks of this handle
   int32_t Bd, kb, kp, m;
   int32_t last_len;
-  int32_t threads;
+  int32_t threads;       // CTA size of the select variants (32 elements per thread)
+  int32_t apply_threads; // CTA size of the apply kernel (two passes per block from B_d 2048)
   bool vec;             // 16-byte vector path usable (B_d % 8 == 0)
   bool persistent;      // bulk-copy pipelined kernels usable (B_d % 32 == 0)
   int32_t variant;      // select kernel: 0 warp per block, 1 CTA per block, 2 persistent CTAs
@@ -91,6 +92,7 @@ int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
   h->m = m;
   h->last_len = (int32_t)(h->d - (block_count - 1) * Bd);
   h->threads = pick_threads(Bd);
+  h->apply_threads = h->threads >= 64 ? h->threads / 2 : h->threads;
   h->vec = (Bd % 8) == 0;
   h->persistent = false;
   h->variant = 0;
@@ -98,7 +100,7 @@ int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
   h->off_window = h->off_codes + round_up((h->d + 1) / 2, 256);
   h->bytes = h->off_window + 4 * block_count * (int64_t)m * kp;
   h->select_smem = mua::select_smem_bytes(h->threads, Bd, kp, m);
-  h->apply_smem = mua::apply_smem_bytes(h->threads, Bd, kp, m);
+  h->apply_smem = mua::apply_smem_bytes(h->apply_threads, Bd, kp, m);
   h->update_split = kDefaultUpdateSplit;
   *out = h;
   return MUA_OK;
@@ -245,7 +247,7 @@ int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float 
                            vhat, &A);
   if (rc != MUA_OK) return rc;
   const cudaError_t e =
-      mua::launch_apply(A, h->threads, h->vec, h->apply_smem, static_cast<cudaStream_t>(stream));
+      mua::launch_apply(A, h->apply_threads, h->vec, h->apply_smem, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "apply kernel launch");
   return MUA_OK;
 }

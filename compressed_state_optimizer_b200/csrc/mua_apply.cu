@@ -1,6 +1,6 @@
 // Stage kernel 2 of the MicroAdam step ([MicroAdam ¶1] = paragraph 1 of
 // "MicroAdam (Sparse-Gradient Adaptive Optimization with Quantized Error
-// Feedback)"), one CTA per block of B_d parameters, once the select kernel has
+// Feedback)"), one CTA per block of B_d parameters (in passes of 32 T elements), once the select kernel has
 // written every block's new window row and the global (delta_{t+1},
 // Delta_{t+1}) is final:
 //   e_{t+1} = Q(a_t, delta_{t+1}, Delta_{t+1}): a_t is recomputed bit for bit
@@ -59,13 +59,20 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
   const float Dn = __uint_as_float(A.hdr[A.pair_next + 1]);
   const float inv16 =
       (Dn == dn) ? 0.0f : __fmul_rn(__fdiv_rn(15.0f, __fsub_rn(Dn, dn)), 65536.0f);
-  const uint64_t grp0 = (uint64_t)(G.base_index + start) >> 3;  // VEC: start % 8 == 0
   const char* lvb = reinterpret_cast<const char*>(s_lv);
+  // The block in passes of kChunks * 8 * T elements (the first pass's loads
+  // were issued above).
+  constexpr int kPass = kChunks * kChunk * T;
+  for (int base = 0; base < L; base += kPass) {
+  const int Lp = L - base;  // elements from this pass's start to the block's end
+  if (base > 0) load_block<T, VEC>(A.grads, A.codes, start + base, Lp, tid, gv, cv);
+  const uint64_t grp0 = (uint64_t)(G.base_index + start + base) >> 3;  // VEC: multiple of 8
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
     const int e0 = elem_index<T>(c, tid, 0);
-    if (e0 >= L) continue;
-    const uint32_t selbits = (sel[e0 >> 5] >> (e0 & 31)) & 0xFFu;
+    if (e0 >= Lp) continue;
+    const int eb = base + e0;  // block-relative index of the chunk's first element
+    const uint32_t selbits = (sel[eb >> 5] >> (eb & 31)) & 0xFFu;
     uint32_t pack = 0u;
     if (VEC) {
       const uint64_t grp = grp0 + (uint64_t)(c * T + tid);
@@ -92,7 +99,7 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
         pack |= (e + 1 <= 4 ? (hi1 >> (12 - 4 * e)) : (hi1 << (4 * e - 12))) & (0xFu << (4 * e + 4));
       }
     } else {
-      const int64_t gidx = G.base_index + start + e0;
+      const int64_t gidx = G.base_index + start + eb;
       const uint64_t ga = (uint64_t)gidx >> 3;
       const uint4 xa = philox4x32_10((uint32_t)ga, (uint32_t)(ga >> 32), A.t_lo, A.t_hi, A.keys);
       const uint4 xb =
@@ -111,14 +118,15 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
         pack |= ((hi >> 16) & 0xFu) << (4 * e);
       }
     }
-    uint8_t* cdst = A.codes + ((start + e0) >> 1);
-    if (VEC && e0 + kChunk <= L) {
+    uint8_t* cdst = A.codes + ((start + eb) >> 1);
+    if (VEC && e0 + kChunk <= Lp) {
       *reinterpret_cast<uint32_t*>(cdst) = pack;
     } else {
-      const int nval = min(kChunk, L - e0);  // nibbles past the block's end stay 0
+      const int nval = min(kChunk, Lp - e0);  // nibbles past the block's end stay 0
       if (nval < kChunk) pack &= (1u << (4 * nval)) - 1u;
       for (int e = 0; e < nval; e += 2) cdst[e >> 1] = (uint8_t)(pack >> (4 * e));
     }
+  }
   }
   if (!update_in_select(A, j)) {  // (6) AdamStats update of block j
     __syncthreads();

@@ -459,11 +459,22 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   }
   __syncthreads();
 
-  // Union rank of each mask word (T >= Wn: one word per thread).
-  const uint32_t pc = (tid < Wn) ? (uint32_t)__popc(mask[tid]) : 0u;
+  // Union rank of each mask word (thread tid: words q tid .. q tid + q - 1).
+  const int q = (Wn + T - 1) / T;
+  uint32_t pc = 0u;
+  for (int i = 0; i < q; ++i) {
+    const int w = q * tid + i;
+    if (w < Wn) pc += (uint32_t)__popc(mask[w]);
+  }
   uint32_t U;
-  const uint32_t incl = block_scan_1bar<T, uint32_t>(pc, scan, U);
-  if (tid < Wn) wpre[tid] = (uint16_t)(incl - pc);
+  uint32_t run = block_scan_1bar<T, uint32_t>(pc, scan, U) - pc;
+  for (int i = 0; i < q; ++i) {
+    const int w = q * tid + i;
+    if (w < Wn) {
+      wpre[w] = (uint16_t)run;
+      run += (uint32_t)__popc(mask[w]);
+    }
+  }
   __syncthreads();
 
   // Each staged entry: index -> union rank (U <= 15360, so a rank never equals
