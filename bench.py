@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama2_7b",
-                    help="llama2_7b | flat_134m | flat_1m | bert_base | flat_1g_m<m>")
+                    help="llama2_7b | flat_134m | flat_1m | bert_base | bert_base_<B_d> | flat_1g_m<m>")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--update-split", type=int, default=None,
@@ -66,6 +66,9 @@ def get_workload(name):
         return W.flat_small()
     if name == "bert_base":
         return W.bert_base()
+    m = re.fullmatch(r"bert_base_(\d+)", name)
+    if m:
+        return W.bert_base(int(m.group(1)))
     m = re.fullmatch(r"flat_1g_m(\d+)", name)
     if m:
         return W.flat_1g(int(m.group(1)))

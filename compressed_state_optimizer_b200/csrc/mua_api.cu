@@ -264,6 +264,10 @@ int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float l
 int mua_set_select_variant(mua_t h, int32_t variant) {
   if (!h || variant < 0 || variant > 2) return MUA_ERR_ARG;
   if (variant == 2 && !((h->Bd % 32) == 0 && h->nb >= 2)) return MUA_ERR_UNSUPPORTED;
+  // The CTA shapes hold the update's shared memory too (and variant 2 a copy
+  // of the block): it must fit one CTA's 227 KB beside the static arrays.
+  const uint32_t stage = variant == 2 ? ((2u * (uint32_t)h->Bd + (uint32_t)h->Bd / 2u + 127u) & ~127u) : 0u;
+  if (variant != 0 && h->select_smem + stage > 227u * 1024u - 8u * 1024u) return MUA_ERR_UNSUPPORTED;
   h->variant = variant;
   return MUA_OK;
 }

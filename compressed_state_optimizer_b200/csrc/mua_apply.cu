@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
 template <int T>
 cudaError_t launch_t(const StepArgs& args, bool vec, uint32_t smem, cudaStream_t stream) {
   auto kern = vec ? mua_apply_kernel<T, true> : mua_apply_kernel<T, false>;
-  if (smem > 48 * 1024) {
+  if (smem > 32 * 1024) {  // opt in well below 48 KB: static arrays count too
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

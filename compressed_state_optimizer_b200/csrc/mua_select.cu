@@ -625,7 +625,7 @@ cudaError_t launch_t(const StepArgs& args, bool vec, bool persistent, uint32_t s
     return cudaGetLastError();
   }
   auto kern = vec ? mua_select_kernel<T, true> : mua_select_kernel<T, false>;
-  if (smem > 48 * 1024) {
+  if (smem > 32 * 1024) {  // opt in well below 48 KB: static arrays count too
     const cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

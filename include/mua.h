@@ -185,6 +185,8 @@ int mua_set_update_split(mua_t h, int32_t split);
  *   2 persistent CTAs streaming each next block into shared memory with
  *     bulk copies (needs B_d % 32 == 0 and at least 2 blocks, else
  *     MUA_ERR_UNSUPPORTED).
+ * Variants 1 and 2 also return MUA_ERR_UNSUPPORTED when one block's select
+ * and AdamStats working set does not fit one CTA's shared memory.
  * Host only; MUA_ERR_ARG for other values.
  */
 int mua_set_select_variant(mua_t h, int32_t variant);

@@ -122,6 +122,7 @@ def test_flat_2p20_through_mua_step():
     (3 * 16384, 16384, 164, 37, 40, "normal"),       # m = 37 (the m_max bound)
     (64 * 33, 64, 64, 12, 12, "normal"),             # k_b = B_d: every entry kept
     (2 * 16384 + 3000, 16384, 1536, 10, 12, "t3"),   # largest window: m * kp = 15360
+    (2 * 16384 + 100, 16384, 164, 20, 22, "normal"),  # apply smem just under 48 KB
 ])
 def test_shapes(d, Bd, kb, m, steps, kind):
     run_parity(d, Bd, kb, m, steps, kind=kind)
