@@ -565,7 +565,7 @@ cudaError_t launch_apply(const StepArgs& args, int threads, bool vec, uint32_t s
                          cudaStream_t stream);
 uint32_t select_smem_bytes(int threads, int Bd, int kp, int m);
 cudaError_t launch_select_warp(const StepArgs& args, bool vec, cudaStream_t stream);
-uint32_t select_warp_smem_bytes();
+uint32_t select_warp_smem_bytes(int Bd);
 uint32_t apply_smem_bytes(int threads, int Bd, int kp, int m);
 
 }  // namespace mua

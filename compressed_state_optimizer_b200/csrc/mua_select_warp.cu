@@ -12,10 +12,11 @@
 // blocks are in flight per SM and memory latency hides behind the others.
 //
 // Exact Top-k:
-//  * candidate path (blocks of 4096 to 16384 entries): 512 sample keys (64
+//  * candidate path (blocks of 1024 to 32768 entries): 512 sample keys (64
 //    chunks of 8 spread over the block), each lane's top-2, a warp sort of
-//    those 64 values -> tau_lo (aiming at ~2.5k candidates); one streaming
-//    pass (lane l holds elements 256 s + 8 l .. + 7 of step s) appends every
+//    those 64 values -> tau_lo (aiming at ~2.5k candidates over the block);
+//    one streaming pass (lane l holds elements 256 s + 8 l .. + 7 of step s)
+//    appends every
 //    |a| >= tau_lo to the lane's own strided region of the list, with no
 //    cross-lane step, and folds the rest into the residual min/max; an exact
 //    warp radix select on the list (8-bit digits from the highest bit where
@@ -23,9 +24,10 @@
 //    entries are marked in a bitmask of the block (ties at the threshold by a
 //    lowest-index merge of the lanes' regions, each already in index order)
 //    and a popcount prefix of the mask gives each its place in the row;
-//  * fallback (small blocks, or fewer than k / more than kLaneCap candidates
-//    in a lane): exact radix select on all keys by streaming passes over the
-//    block (it is in L2 by then), 8 bits per pass, then one placing pass.
+//  * fallback (blocks under 1024 entries, k > L/8, too few candidates after
+//    the retry, or a lane that dropped a key at or above the threshold):
+//    exact radix select on all keys by streaming passes over the block (it
+//    is in L2 by then), 8 bits per pass, then one placing pass.
 // HBM traffic per parameter: 2 B gradient + 0.5 B codes read; per selected
 // entry 4 B written.
 #include "mua_kernels.cuh"
@@ -36,19 +38,23 @@ namespace {
 constexpr int kWarps = 8;         // warps (= blocks in flight) per CTA
 constexpr int kWarpCap = 1024;    // candidate list entries per warp
 constexpr int kLaneCap = kWarpCap / 32;  // entries per lane region
-constexpr int kSelMaskWords = 512;       // selection bitmask: blocks of up to 16384
 constexpr int kUnroll = 4;        // 256-element steps loaded ahead
 
+// MASKW: words of the selection bitmask, which covers one block (512 for
+// blocks of up to 16384 entries, 1024 up to 32768).
+template <int MASKW>
 struct WarpSmem {
   uint32_t bits[kWarpCap];  // a_t bits; lane l's i-th candidate at [32 i + l]
   uint16_t idx[kWarpCap];   // its block-relative index
-  uint32_t hist[256];       // radix histogram, then the mask's u16 word prefix
-  uint32_t mask[kSelMaskWords];
+  uint32_t hist[MASKW / 2 > 256 ? MASKW / 2 : 256];  // radix histogram, then the
+                                                     // mask's u16 word prefix
+  uint32_t mask[MASKW];
 };
 
+template <int MASKW>
 struct CtaSmem {
   float levels[16];
-  WarpSmem w[kWarps];
+  WarpSmem<MASKW> w[kWarps];
 };
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
@@ -226,10 +232,10 @@ __device__ __forceinline__ void warp_radix(int hi, uint32_t prefix, int k, uint3
   need = krem;
 }
 
-template <bool VEC>
+template <bool VEC, int MASKW>
 __global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const StepArgs A) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  CtaSmem& S = *reinterpret_cast<CtaSmem*>(dyn);
+  CtaSmem<MASKW>& S = *reinterpret_cast<CtaSmem<MASKW>*>(dyn);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const Geometry& G = A.g;
   {
@@ -240,7 +246,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const S
   __syncthreads();  // the only CTA barrier: the level table
   const int j = blockIdx.x * kWarps + wid;
   if (j >= G.nb) return;
-  WarpSmem& W = S.w[wid];
+  WarpSmem<MASKW>& W = S.w[wid];
   const float* lv = S.levels;
   const int64_t start = (int64_t)j * G.Bd;
   const int L = (j == G.nb - 1) ? G.last_len : G.Bd;
@@ -252,7 +258,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const S
   bool done = false;
 
   // ---------------- candidate path
-  if (L >= 4096 && L <= 32 * kSelMaskWords && 8 * k <= L) {
+  if (L >= 1024 && L <= 32 * MASKW && 8 * k <= L) {
     // 512 samples: 64 chunks of 8, chunk c at element (c * (L / 64)) & ~7.
     const int cstride = (L / 64) & ~7;
     uint32_t t1 = 0u, t2 = 0u;  // this lane's two largest sample keys
@@ -296,7 +302,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const S
         }
       }
     }
-    const int r = min(63, (5 * k + 63) / 64 - 1);  // ~2.5k of 32x as many elements
+    // rank of tau_lo among the 64: ~2.5k candidates expected over the block
+    const int r = min(63, (int)((1280 * (int64_t)k + L - 1) / L) - 1);
     const uint32_t tl0 = __shfl_sync(0xFFFFFFFFu, v0, r >> 1);
     const uint32_t tl1 = __shfl_sync(0xFFFFFFFFu, v1, r >> 1);
     const uint32_t tau_first = (r & 1) ? tl1 : tl0;
@@ -409,16 +416,18 @@ __global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const S
         }
       }
       __syncwarp();
-      // u16 exclusive popcount prefix of the mask words (lane l: words 16 l ..)
+      // u16 exclusive popcount prefix of the mask words (lane l: words
+      // MASKW/32 l ..)
       uint16_t* wpre = reinterpret_cast<uint16_t*>(W.hist);
       {
-        const int w0 = 16 * lane;
+        constexpr int kWpl = MASKW / 32;
+        const int w0 = kWpl * lane;
         uint32_t c = 0u;
 #pragma unroll
-        for (int w = 0; w < 16; ++w) c += (w0 + w < wn) ? (uint32_t)__popc(W.mask[w0 + w]) : 0u;
+        for (int w = 0; w < kWpl; ++w) c += (w0 + w < wn) ? (uint32_t)__popc(W.mask[w0 + w]) : 0u;
         uint32_t run = warp_incl_scan(c, lane) - c;
 #pragma unroll
-        for (int w = 0; w < 16; ++w) {
+        for (int w = 0; w < kWpl; ++w) {
           if (w0 + w < wn) {
             wpre[w0 + w] = (uint16_t)run;
             run += (uint32_t)__popc(W.mask[w0 + w]);
@@ -528,11 +537,15 @@ __global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const S
 
 }  // namespace
 
-uint32_t select_warp_smem_bytes() { return (uint32_t)sizeof(CtaSmem); }
+uint32_t select_warp_smem_bytes(int Bd) {
+  return Bd <= 16384 ? (uint32_t)sizeof(CtaSmem<512>) : (uint32_t)sizeof(CtaSmem<1024>);
+}
 
 cudaError_t launch_select_warp(const StepArgs& args, bool vec, cudaStream_t stream) {
-  auto kern = vec ? mua_select_warp_kernel<true> : mua_select_warp_kernel<false>;
-  const uint32_t smem = select_warp_smem_bytes();
+  const bool big = args.g.Bd > 16384;
+  auto kern = big ? (vec ? mua_select_warp_kernel<true, 1024> : mua_select_warp_kernel<false, 1024>)
+                  : (vec ? mua_select_warp_kernel<true, 512> : mua_select_warp_kernel<false, 512>);
+  const uint32_t smem = select_warp_smem_bytes(args.g.Bd);
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
