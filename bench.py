@@ -51,12 +51,20 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--update-split", type=int, default=None,
                     help="eighths of the blocks whose parameter update runs in the select kernel")
+    ap.add_argument("--wd", type=float, default=None,
+                    help="weight decay instead of the workload's (AdamW-style, every parameter)")
     ap.add_argument("--cpu-sample", type=int, default=1 << 23,
                     help="parameters in the oracle's bounded sample")
     return ap.parse_args()
 
 
-def get_workload(name):
+def get_workload(name, wd=None):
+    import dataclasses
+    w = _named_workload(name)
+    return w if wd is None else dataclasses.replace(w, wd=wd)
+
+
+def _named_workload(name):
     from compressed_state_optimizer_b200 import workloads as W
     if name == "llama2_7b":
         return W.llama2_7b()
@@ -219,7 +227,7 @@ def cpu_baseline(w, sample: int, max_seconds: float = 12.0, min_steps: int = 2):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = get_workload(args.workload)
+    w = get_workload(args.workload, args.wd)
     n = min(args.cpu_sample, w.d)
     import oracle
     from compressed_state_optimizer_b200 import workloads as W
@@ -241,7 +249,7 @@ def run_reference(args, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": w.name, "d": w.d, "B_d": w.Bd, "k_b": w.kb, "m": w.m, "b": 4,
+            "config": {"workload": w.name, "d": w.d, "B_d": w.Bd, "k_b": w.kb, "m": w.m, "b": 4, "wd": w.wd,
                        "sample_params": n, "l2": "host run"},
             "cpu_baseline": {"value": value, "unit": "Gparams/s", "cores": 1, "kind": "oracle",
                              "sample": f"first {n} parameters of {w.name} per step"},
@@ -258,7 +266,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = get_workload(args.workload)
+    w = get_workload(args.workload, args.wd)
     mo = MicroAdam(w.d, block_size=w.Bd, k_per_block=w.kb, window=w.m,
                    shard=None if world == 1 else sharding.shard_blocks(w.d, w.Bd, rank, world))
     if args.update_split is not None:
@@ -349,7 +357,7 @@ def run_ours(args, rank, world, local_rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": {"workload": w.name, "d": w.d, "B_d": w.Bd, "k_b": w.kb, "m": w.m,
+            "config": {"workload": w.name, "d": w.d, "B_d": w.Bd, "k_b": w.kb, "m": w.m, "wd": w.wd,
                        "b": 4, "grads": w.grad, "parallelism": f"blocks sharded over {world}"
                        if world > 1 else "single GPU",
                        "l2": "inputs (params+grads+state ~47 GB) larger than L2"},
