@@ -153,12 +153,17 @@ def gpu_id(dev) -> str:
         return str(dev.index or 0)
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(csrc: str | None = None) -> str:
+    """Hash of the CUDA sources' code (// comments and blank lines dropped, so
+    a comment edit keeps a profile taken on the same code valid)."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "compressed_state_optimizer_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "compressed_state_optimizer_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
         if f.endswith((".cu", ".cuh")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+            for line in open(os.path.join(csrc, f), encoding="utf-8"):
+                code = re.sub(r"//.*", "", line).rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

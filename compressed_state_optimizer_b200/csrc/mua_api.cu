@@ -5,10 +5,12 @@
 //
 // A handle holds geometry only. mua_step enqueues, on the caller's stream:
 //   1. an 8-byte memset of the (-delta_{t+1}, Delta_{t+1}) accumulator pair,
-//   2. the select kernel (one CTA per block; also updates the parameters of
-//      the blocks with (j & 7) < update_split),
-//   3. the apply kernel (one CTA per block, reverse block order so the tail of
-//      the select kernel's reads is still in L2; updates the other blocks).
+//   2. the select kernel: by default one warp per block (mua_select_warp.cu);
+//      the CTA shapes of mua_select.cu (variants 1, 2) can also update the
+//      parameters of the blocks with (j & 7) < update_split,
+//   3. the apply kernel (one CTA of half the select CTA's threads per block,
+//      reverse block order so the tail of the select kernel's reads is still
+//      in L2): codec, then the AdamStats update of the remaining blocks.
 // Everything the kernels need per step (beta^r weights, bias corrections,
 // Philox round keys) is computed here in fp64 and rounded once to fp32 /
 // uint32 before launch.
