@@ -66,6 +66,11 @@ def lib() -> ctypes.CDLL:
         L.mua_oracle_step.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P,
                                       f64, f64, f64, f64, f64, i64, u64, P, P, P]
         L.mua_oracle_step.restype = ctypes.c_int
+        L.mua_oracle_step_seg.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P,
+                                          f64, f64, f64, f64, f64, i64, u64, P, P, P]
+        L.mua_oracle_step_seg.restype = ctypes.c_int
+        L.mua_oracle_num_blocks.argtypes = [P, i32, i32]
+        L.mua_oracle_num_blocks.restype = i64
         _lib = L
     return _lib
 
@@ -131,6 +136,8 @@ class OracleState:
     scal   float32[2]         (delta, Delta)
     G_idx  int16[m, n_b, k_b] block-relative indices of the window rows (-1 empty)
     G_val  uint16[m, n_b, k_b] bf16 bits of the window values
+    segs   int64[n] segment (tensor) lengths, blocks cut per segment; one
+           segment of length d is the flat cut
     """
     d: int
     Bd: int
@@ -140,24 +147,39 @@ class OracleState:
     scal: np.ndarray
     G_idx: np.ndarray
     G_val: np.ndarray
+    segs: np.ndarray | None = None
 
     @property
     def nb(self) -> int:
-        return (self.d + self.Bd - 1) // self.Bd
+        return self.G_idx.shape[1]
 
     def copy(self) -> "OracleState":
         return OracleState(self.d, self.Bd, self.kb, self.m, self.codes.copy(),
-                           self.scal.copy(), self.G_idx.copy(), self.G_val.copy())
+                           self.scal.copy(), self.G_idx.copy(), self.G_val.copy(),
+                           None if self.segs is None else self.segs.copy())
 
 
-def new_state(d: int, Bd: int, kb: int, m: int) -> OracleState:
-    """The initial state: e_0 = 0 with delta = Delta = 0 and an empty window."""
-    nb = (d + Bd - 1) // Bd
+def num_blocks(segs, Bd: int) -> int:
+    segs = np.ascontiguousarray(segs, dtype=np.int64)
+    return int(lib().mua_oracle_num_blocks(_ptr(segs), segs.size, Bd))
+
+
+def new_state(d: int, Bd: int, kb: int, m: int, segments=None) -> OracleState:
+    """The initial state: e_0 = 0 with delta = Delta = 0 and an empty window.
+    ``segments``: tensor lengths summing to d, blocks cut per tensor."""
+    segs = None
+    if segments is not None:
+        segs = np.ascontiguousarray(segments, dtype=np.int64)
+        assert int(segs.sum()) == d and np.all(segs > 0)
+        nb = num_blocks(segs, Bd)
+    else:
+        nb = (d + Bd - 1) // Bd
     return OracleState(d, Bd, kb, m,
                        codes=np.zeros((d + 1) // 2, dtype=np.uint8),
                        scal=np.zeros(2, dtype=np.float32),
                        G_idx=np.full((m, nb, kb), -1, dtype=np.int16),
-                       G_val=np.zeros((m, nb, kb), dtype=np.uint16))
+                       G_val=np.zeros((m, nb, kb), dtype=np.uint16),
+                       segs=segs)
 
 
 def step(st: OracleState, p: np.ndarray, g_bits: np.ndarray, *, lr: float, beta1: float,
@@ -176,10 +198,17 @@ def step(st: OracleState, p: np.ndarray, g_bits: np.ndarray, *, lr: float, beta1
     if want_stats:
         stats = tuple(np.zeros(st.d, dtype=np.float64) for _ in range(3))
     f = lambda v: float(np.float32(v))  # noqa: E731  (the fp32 value the kernels see)
-    rc = lib().mua_oracle_step(st.d, st.Bd, st.kb, st.m, _ptr(p), _ptr(g_bits),
-                               _ptr(st.codes), _ptr(st.scal), _ptr(st.G_idx),
-                               _ptr(st.G_val), f(lr), f(beta1), f(beta2), f(eps), f(wd),
-                               t, seed, *(_ptr(s) for s in (stats or (None,) * 3)))
+    if st.segs is None:
+        rc = lib().mua_oracle_step(st.d, st.Bd, st.kb, st.m, _ptr(p), _ptr(g_bits),
+                                   _ptr(st.codes), _ptr(st.scal), _ptr(st.G_idx),
+                                   _ptr(st.G_val), f(lr), f(beta1), f(beta2), f(eps), f(wd),
+                                   t, seed, *(_ptr(s) for s in (stats or (None,) * 3)))
+    else:
+        rc = lib().mua_oracle_step_seg(_ptr(st.segs), st.segs.size, st.Bd, st.kb, st.m,
+                                       _ptr(p), _ptr(g_bits), _ptr(st.codes), _ptr(st.scal),
+                                       _ptr(st.G_idx), _ptr(st.G_val), f(lr), f(beta1),
+                                       f(beta2), f(eps), f(wd), t, seed,
+                                       *(_ptr(s) for s in (stats or (None,) * 3)))
     if rc != 0:
         raise ValueError("oracle step rejected its arguments")
     return stats

@@ -34,8 +34,8 @@
  *  - update u = m_hat / (eps + sqrt(v_hat)); decoupled weight decay
  *    p <- p*(1 - lr*wd) is applied to every coordinate before the update.
  *  - delta, Delta are global over the flat d-vector; blocks are cut over
- *    that vector; a ragged last block of length L keeps
- *    k = ceil(L*k_b/B_d) entries.
+ *    that vector, or, for a tensor list, over each tensor (segment) in turn;
+ *    a ragged last block of length L keeps k = ceil(L*k_b/B_d) entries.
  */
 #include <math.h>
 #include <stdint.h>
@@ -189,13 +189,29 @@ int64_t mua_oracle_block_k(int64_t L, int32_t Bd, int32_t kb) {
 /*                       sum_r b1^r |V_r|; zero where no window entry.      */
 /* Returns 0, or -1 on bad arguments / allocation failure.                  */
 /* ---------------------------------------------------------------------- */
-int mua_oracle_step(int64_t d, int32_t Bd, int32_t kb, int32_t m, float* p,
-                    const uint16_t* g, uint8_t* codes, float* scal, int16_t* G_idx,
-                    uint16_t* G_val, double lr, double beta1, double beta2, double eps,
-                    double wd, int64_t t, uint64_t seed, double* mhat, double* vhat,
-                    double* mabs) {
-    if (d < 1 || Bd < 1 || Bd > 32766 || kb < 1 || kb > Bd || m < 1 || t < 1) return -1;
-    const int64_t nb = (d + Bd - 1) / Bd;
+/* Number of blocks when the d-vector is the concatenation of n_seg segments
+ * (tensors) of the given lengths, each cut into its own blocks of B_d with a
+ * ragged last block; one segment of length d is the plain flat cut. */
+int64_t mua_oracle_num_blocks(const int64_t* seg, int32_t n_seg, int32_t Bd) {
+    int64_t nb = 0;
+    for (int32_t s = 0; s < n_seg; ++s) nb += (seg[s] + Bd - 1) / Bd;
+    return nb;
+}
+
+/* One MicroAdam step [MicroAdam ¶1] over the concatenation of n_seg segments
+ * of lengths seg[0..n_seg) (d = their sum), blocks cut per segment. */
+int mua_oracle_step_seg(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, int32_t m,
+                        float* p, const uint16_t* g, uint8_t* codes, float* scal,
+                        int16_t* G_idx, uint16_t* G_val, double lr, double beta1,
+                        double beta2, double eps, double wd, int64_t t, uint64_t seed,
+                        double* mhat, double* vhat, double* mabs) {
+    if (n_seg < 1 || Bd < 1 || Bd > 32766 || kb < 1 || kb > Bd || m < 1 || t < 1) return -1;
+    int64_t d = 0;
+    for (int32_t s = 0; s < n_seg; ++s) {
+        if (seg[s] < 1) return -1;
+        d += seg[s];
+    }
+    const int64_t nb = mua_oracle_num_blocks(seg, n_seg, Bd);
     const float delta_t = scal[0], Delta_t = scal[1];
 
     float* a = (float*)malloc(sizeof(float) * (size_t)d);
@@ -204,9 +220,23 @@ int mua_oracle_step(int64_t d, int32_t Bd, int32_t kb, int32_t m, float* p,
     double* z2 = (double*)calloc((size_t)d, sizeof(double));
     double* za = (double*)calloc((size_t)d, sizeof(double));
     uint8_t* touched = (uint8_t*)calloc((size_t)d, 1);
-    if (!a || !order || !z1 || !z2 || !za || !touched) {
+    int64_t* bstart = (int64_t*)malloc(sizeof(int64_t) * (size_t)nb);
+    int64_t* blen = (int64_t*)malloc(sizeof(int64_t) * (size_t)nb);
+    if (!a || !order || !z1 || !z2 || !za || !touched || !bstart || !blen) {
         free(a); free(order); free(z1); free(z2); free(za); free(touched);
+        free(bstart); free(blen);
         return -1;
+    }
+    /* The blocks, in order: segment by segment, B_d at a time. */
+    {
+        int64_t j = 0, off = 0;
+        for (int32_t s = 0; s < n_seg; ++s) {
+            for (int64_t b = 0; b < seg[s]; b += Bd, ++j) {
+                bstart[j] = off + b;
+                blen[j] = (seg[s] - b < Bd) ? (seg[s] - b) : Bd;
+            }
+            off += seg[s];
+        }
     }
 
     /* (1) a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t). */
@@ -223,8 +253,8 @@ int mua_oracle_step(int64_t d, int32_t Bd, int32_t kb, int32_t m, float* p,
      * (3) the selected entries of a_t are set to zero. */
     const int64_t row = t % m;
     for (int64_t j = 0; j < nb; ++j) {
-        const int64_t start = j * (int64_t)Bd;
-        const int64_t L = (d - start < Bd) ? (d - start) : Bd;
+        const int64_t start = bstart[j];
+        const int64_t L = blen[j];
         const int64_t k = mua_oracle_block_k(L, Bd, kb);
         for (int64_t q = 0; q < L; ++q) {
             order[q].key = bits_from_f32(a[start + q]) & 0x7FFFFFFFu;
@@ -273,7 +303,7 @@ int mua_oracle_step(int64_t d, int32_t Bd, int32_t kb, int32_t m, float* p,
             const uint16_t* rv = G_val + (rr * nb + j) * kb;
             for (int64_t s = 0; s < kb; ++s) {
                 if (ri[s] < 0) continue;
-                const int64_t q = j * (int64_t)Bd + ri[s];
+                const int64_t q = bstart[j] + ri[s];
                 const double V = (double)mua_oracle_bf16_to_f32(rv[s]);
                 z1[q] += w1 * V;
                 z2[q] += w2 * (V * V);
@@ -300,5 +330,17 @@ int mua_oracle_step(int64_t d, int32_t Bd, int32_t kb, int32_t m, float* p,
     }
 
     free(a); free(order); free(z1); free(z2); free(za); free(touched);
+    free(bstart); free(blen);
     return 0;
+}
+
+/* The flat cut: one segment of length d. */
+int mua_oracle_step(int64_t d, int32_t Bd, int32_t kb, int32_t m, float* p,
+                    const uint16_t* g, uint8_t* codes, float* scal, int16_t* G_idx,
+                    uint16_t* G_val, double lr, double beta1, double beta2, double eps,
+                    double wd, int64_t t, uint64_t seed, double* mhat, double* vhat,
+                    double* mabs) {
+    if (d < 1) return -1;
+    return mua_oracle_step_seg(&d, 1, Bd, kb, m, p, g, codes, scal, G_idx, G_val, lr, beta1,
+                               beta2, eps, wd, t, seed, mhat, vhat, mabs);
 }

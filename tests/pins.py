@@ -407,9 +407,88 @@ def check_block_locality():
         assert np.array_equal(part.G_val[1 % m, 0], full.G_val[1 % m, j])
 
 
+# --------------------------------------------------------------- tensor lists
+def _seg_blocks(segs, Bd):
+    """(start, length) of every block when each tensor is cut on its own."""
+    out, off = [], 0
+    for n in segs:
+        out += [(off + b, min(Bd, n - b)) for b in range(0, n, Bd)]
+        off += n
+    return out
+
+
+def check_segmented_topk_minmax_step1():
+    """A tensor list cut per tensor: at t = 1 each tensor's blocks (its own
+    ragged last block included) hold numpy's stable arg-sort of |g| inside the
+    block, k_j = ceil(L_j k_b / B_d) entries; delta_2, Delta_2 are numpy's min
+    and max of the residual over all tensors [MicroAdam ¶1]."""
+    Bd, kb, m = 256, 5, 2
+    segs = [3 * 256 + 40, 100, 256, 2 * 256 + 2]
+    d = sum(segs)
+    g_bits = normal_bf16(d, 31)
+    st = oracle.new_state(d, Bd, kb, m, segments=segs)
+    p = np.zeros(d, dtype=np.float32)
+    oracle.step(st, p, g_bits, lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, wd=0.0, t=1, seed=3)
+    a = f32_of_bits(g_bits).copy()
+    blocks = _seg_blocks(segs, Bd)
+    assert st.nb == len(blocks)
+    for j, (b0, L) in enumerate(blocks):
+        rows = topk_rows_numpy(a[b0:b0 + L], Bd, kb)[0]
+        k = rows.size
+        assert np.array_equal(st.G_idx[1 % m, j, :k], rows), j
+        assert np.all(st.G_idx[1 % m, j, k:] == -1), j
+        assert np.array_equal(f32_of_bits(st.G_val[1 % m, j, :k]), a[b0 + rows])
+    for j, (b0, L) in enumerate(blocks):
+        k = -(-L * kb // Bd)
+        a[b0 + st.G_idx[1 % m, j, :k].astype(np.int64)] = 0.0
+    assert st.scal[0] == np.min(a) and st.scal[1] == np.max(a)
+
+
+def check_segmented_update_support():
+    """With a tensor list, the update touches exactly the window's indices
+    placed at their tensor's block starts (wd = 0) [MicroAdam ¶1, ¶5]."""
+    Bd, kb, m = 128, 4, 3
+    segs = [300, 128, 77, 250]
+    d = sum(segs)
+    st = oracle.new_state(d, Bd, kb, m, segments=segs)
+    p = np.random.default_rng(4).standard_normal(d).astype(np.float32)
+    blocks = _seg_blocks(segs, Bd)
+    for t in range(1, 6):
+        before = p.copy()
+        oracle.step(st, p, normal_bf16(d, 60 + t), lr=1e-2, beta1=0.9, beta2=0.999, eps=1e-8,
+                    wd=0.0, t=t, seed=9)
+        want = set()
+        for r in range(min(t, m)):
+            for j, (b0, _) in enumerate(blocks):
+                idx = st.G_idx[(t - r) % m, j]
+                want.update(int(b0 + i) for i in idx[idx >= 0])
+        assert set(np.flatnonzero(p != before).tolist()) == want, t
+
+
+def check_segmented_whole_blocks_equal_flat():
+    """Tensors that are whole multiples of B_d are cut exactly as the flat
+    vector, and so is a single tensor: the states agree bit for bit."""
+    Bd, kb, m = 128, 3, 3
+    for segs in ([5 * 128 + 17], [2 * 128, 128, 3 * 128]):
+        d = sum(segs)
+        flat, seg = oracle.new_state(d, Bd, kb, m), oracle.new_state(d, Bd, kb, m, segments=segs)
+        pf = np.random.default_rng(5).standard_normal(d).astype(np.float32)
+        ps = pf.copy()
+        for t in range(1, 6):
+            g = normal_bf16(d, 80 + t)
+            hyper = dict(lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, wd=0.01, t=t, seed=2)
+            oracle.step(flat, pf, g, **hyper)
+            oracle.step(seg, ps, g, **hyper)
+        for x, y in ((flat.codes, seg.codes), (flat.scal, seg.scal), (flat.G_idx, seg.G_idx),
+                     (flat.G_val, seg.G_val), (pf, ps)):
+            assert np.array_equal(x, y)
+
+
 ALL = [check_philox_vs_torch, check_draw16_mapping, check_draw16_uniform, check_bf16_rne,
        check_topk_step1, check_minmax_step1, check_topk_later_steps, check_dequant_levels,
        check_quant_exact_levels, check_quant_error_bound, check_quant_unbiased,
        check_lemma1_per_realization, check_adamstats_vs_dense_ema, check_closed_form_m1_t1,
        check_reduces_to_adam, functools.partial(check_reduces_to_adam, wd=0.1),
-       check_lemma3_bound, check_update_sparsity, check_block_locality]
+       check_lemma3_bound, check_update_sparsity, check_block_locality,
+       check_segmented_topk_minmax_step1, check_segmented_update_support,
+       check_segmented_whole_blocks_equal_flat]

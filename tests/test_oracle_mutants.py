@@ -79,6 +79,9 @@ MUTANTS = {
     "weight_decay_dropped": (
         "if (wd != 0.0) pq = pq * decay;",
         ";"),
+    "segment_cut_ignored": (
+        "blen[j] = (seg[s] - b < Bd) ? (seg[s] - b) : Bd;",
+        "blen[j] = (d - (off + b) < Bd) ? (d - (off + b)) : Bd;"),
 }
 
 
