@@ -46,7 +46,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama2_7b",
-                    help="llama2_7b | flat_134m | flat_1m | bert_base | bert_base_<B_d> | flat_1g_m<m>")
+                    help="llama2_7b | llama2_7b_per_tensor | flat_134m | flat_1m | bert_base | "
+                         "bert_base_<B_d> | flat_1g_m<m>")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--update-split", type=int, default=None,
@@ -68,6 +69,9 @@ def _named_workload(name):
     from compressed_state_optimizer_b200 import workloads as W
     if name == "llama2_7b":
         return W.llama2_7b()
+    if name == "llama2_7b_per_tensor":
+        import dataclasses
+        return dataclasses.replace(W.llama2_7b(), name="llama2_7b_per_tensor", per_tensor=True)
     if name == "flat_134m":
         return W.flat_134m()
     if name == "flat_1m":
@@ -272,7 +276,10 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     w = get_workload(args.workload, args.wd)
-    mo = MicroAdam(w.d, block_size=w.Bd, k_per_block=w.kb, window=w.m,
+    segs = w.segments()
+    if segs is not None and world > 1:
+        raise SystemExit("the per-tensor cut runs on one GPU")
+    mo = MicroAdam(w.d, block_size=w.Bd, k_per_block=w.kb, window=w.m, segments=segs,
                    shard=None if world == 1 else sharding.shard_blocks(w.d, w.Bd, rank, world))
     if args.update_split is not None:
         mo.set_update_split(args.update_split)
@@ -336,8 +343,11 @@ def run_ours(args, rank, world, local_rank):
     # ---- algorithmic bytes (per launch, this rank's shard)
     lay = mo.layout
     nb = lay.blocks
-    L_last = d_loc - (nb - 1) * w.Bd
-    K = (nb - 1) * w.kb + -(-L_last * w.kb // w.Bd)
+    if segs is None:
+        L_last = d_loc - (nb - 1) * w.Bd
+        K = (nb - 1) * w.kb + -(-L_last * w.kb // w.Bd)
+    else:  # every tensor's blocks, its ragged last one included
+        K = sum((n // w.Bd) * w.kb + -(-(n % w.Bd) * w.kb // w.Bd) for n in segs)
     win = state[lay.window: lay.window + 4 * nb * w.m * lay.row_stride].view(torch.int32)
     U = union_size(win, nb, w.m, lay.row_stride, w.Bd, d_loc, torch)
     rows = min(t, w.m)
@@ -363,6 +373,7 @@ def run_ours(args, rank, world, local_rank):
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "d": w.d, "B_d": w.Bd, "k_b": w.kb, "m": w.m, "wd": w.wd,
+                       "blocks": "per tensor" if segs is not None else "over the flat vector",
                        "b": 4, "grads": w.grad, "parallelism": f"blocks sharded over {world}"
                        if world > 1 else "single GPU",
                        "l2": "inputs (params+grads+state ~47 GB) larger than L2"},

@@ -30,6 +30,8 @@ SIGNATURES = {
     "mua_create": (ctypes.c_int, [_i64, _i32, _i32, _i32, _i32, ctypes.POINTER(_P)]),
     "mua_create_shard": (ctypes.c_int, [_i64, _i32, _i32, _i32, _i32, _i64, _i64,
                                         ctypes.POINTER(_P)]),
+    "mua_create_segmented": (ctypes.c_int, [ctypes.POINTER(_i64), _i32, _i32, _i32, _i32, _i32,
+                                            ctypes.POINTER(_P)]),
     "mua_destroy": (None, [_P]),
     "mua_state_bytes": (_i64, [_P]),
     "mua_state_layout": (ctypes.c_int, [_P, ctypes.POINTER(_i64)]),
@@ -107,19 +109,30 @@ class Layout:
 
 class MicroAdam:
     """One MicroAdam problem: d parameters in blocks of B_d, k_b kept per block,
-    a window of m rows, b = 4 bits (optionally one rank's shard of the blocks).
+    a window of m rows, b = 4 bits (optionally one rank's shard of the blocks,
+    or, with ``segments``, a tensor list whose tensors are cut into blocks one
+    by one; ``d`` must then be their total length).
 
     The optimizer state is a caller-owned ``torch.uint8`` tensor of
     ``state_bytes`` bytes (see :meth:`new_state`), zero at t = 0.
     """
 
     def __init__(self, d: int, block_size: int = 16384, k_per_block: int | None = None,
-                 window: int = 10, bits: int = 4, *, shard: tuple[int, int] | None = None):
+                 window: int = 10, bits: int = 4, *, shard: tuple[int, int] | None = None,
+                 segments=None):
         if k_per_block is None:
             k_per_block = max(1, math.ceil(block_size / 100 - 1e-9))
         lib = library()
         h = ctypes.c_void_p()
-        if shard is None:
+        self.segments = None if segments is None else [int(n) for n in segments]
+        if self.segments is not None:
+            if shard is not None or sum(self.segments) != d:
+                raise ValueError("segments: whole vector only, lengths summing to d")
+            arr = (_i64 * len(self.segments))(*self.segments)
+            _check(lib.mua_create_segmented(arr, len(self.segments), block_size, k_per_block,
+                                            window, bits, ctypes.byref(h)),
+                   "mua_create_segmented")
+        elif shard is None:
             _check(lib.mua_create(d, block_size, k_per_block, window, bits, ctypes.byref(h)),
                    "mua_create")
         else:
@@ -136,7 +149,7 @@ class MicroAdam:
         arr = (ctypes.c_int64 * 6)()
         _check(lib.mua_state_layout(h, arr), "mua_state_layout")
         self.layout = Layout(*[int(x) for x in arr])
-        nb_total = -(-d // block_size)
+        nb_total = self.layout.blocks if self.segments is not None else -(-d // block_size)
         if shard is None:
             self.first_block, self.blocks = 0, nb_total
         else:

@@ -23,6 +23,8 @@
 #include "../../include/mua.h"
 #include "mua_kernels.cuh"
 
+static_assert(mua::kMaxSegments == MUA_MAX_SEGMENTS, "segment table size");
+
 struct mua_ctx {
   int64_t d;            // elements of this handle
   int64_t d_total;      // elements of the whole vector
@@ -38,6 +40,11 @@ struct mua_ctx {
   int64_t off_codes, off_window, bytes;
   uint32_t select_smem, apply_smem;
   int32_t update_split;  // blocks with (j & 7) < split update in the select kernel
+  // Tensor list cut per tensor (n_seg > 0; whole vector, not a shard).
+  int32_t n_seg;
+  int32_t seg_first[mua::kMaxSegments];
+  int64_t seg_start[mua::kMaxSegments];
+  int64_t seg_len[mua::kMaxSegments];
 };
 
 namespace {
@@ -104,6 +111,46 @@ int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
   h->select_smem = mua::select_smem_bytes(h->threads, Bd, kp, m);
   h->apply_smem = mua::apply_smem_bytes(h->apply_threads, Bd, kp, m);
   h->update_split = kDefaultUpdateSplit;
+  h->n_seg = 0;
+  *out = h;
+  return MUA_OK;
+}
+
+int make_segmented(const int64_t* seg_len, int32_t n_seg, int32_t Bd, int32_t kb, int32_t m,
+                   int32_t bits, mua_t* out) {
+  if (!out) return MUA_ERR_ARG;
+  *out = nullptr;
+  if (!seg_len || n_seg < 1) return MUA_ERR_ARG;
+  if (n_seg > mua::kMaxSegments) return MUA_ERR_UNSUPPORTED;
+  int64_t d = 0, nb = 0;
+  bool all8 = true;
+  for (int32_t s = 0; s < n_seg; ++s) {
+    if (seg_len[s] < 1) return MUA_ERR_ARG;
+    if (seg_len[s] & 1) return MUA_ERR_UNSUPPORTED;  // blocks must start on a code byte
+    if (Bd >= 2) nb += (seg_len[s] + Bd - 1) / Bd;
+    all8 = all8 && (seg_len[s] % 8) == 0;
+    d += seg_len[s];
+  }
+  if (nb > 0x7FFFFFFF) return MUA_ERR_UNSUPPORTED;
+  // The flat geometry of the same d and block count checks the other
+  // arguments and sizes the state; the segment table then replaces the cut.
+  mua_t h = nullptr;
+  int rc = make(d, Bd, kb, m, bits, 0, (d + Bd - 1) / Bd, &h);
+  if (rc != MUA_OK) return rc;
+  h->nb = nb;
+  h->bytes = h->off_window + 4 * nb * (int64_t)m * h->kp;
+  h->vec = h->vec && all8;
+  h->n_seg = n_seg;
+  int64_t first = 0, start = 0;
+  for (int32_t s = 0; s < n_seg; ++s) {
+    h->seg_first[s] = (int32_t)first;
+    h->seg_start[s] = start;
+    h->seg_len[s] = seg_len[s];
+    first += (seg_len[s] + Bd - 1) / Bd;
+    start += seg_len[s];
+  }
+  const int64_t last = seg_len[n_seg - 1];
+  h->last_len = (int32_t)(last - ((last + Bd - 1) / Bd - 1) * (int64_t)Bd);
   *out = h;
   return MUA_OK;
 }
@@ -150,6 +197,11 @@ int mua_create(int64_t d, int32_t block_size, int32_t k_per_block, int32_t windo
 int mua_create_shard(int64_t d_total, int32_t block_size, int32_t k_per_block, int32_t window,
                      int32_t bits, int64_t block_begin, int64_t block_count, mua_t* out) {
   return make(d_total, block_size, k_per_block, window, bits, block_begin, block_count, out);
+}
+
+int mua_create_segmented(const int64_t* seg_len, int32_t n_seg, int32_t block_size,
+                         int32_t k_per_block, int32_t window, int32_t bits, mua_t* out) {
+  return make_segmented(seg_len, n_seg, block_size, k_per_block, window, bits, out);
 }
 
 void mua_destroy(mua_t h) { delete h; }
@@ -205,6 +257,12 @@ static int fill_args(mua_t h, float* params, const uint16_t* grads, void* state,
   A.update_split = (h->variant == 0) ? 0 : h->update_split;
   // Exact for e < 2^16: (2^32 mod kp) < kp and e * kp < 2^31 keep the error below 1/kp.
   A.kp_recip = (uint32_t)(((1ull << 32) + (uint64_t)h->kp - 1) / (uint64_t)h->kp);
+  A.n_seg = h->n_seg;
+  for (int32_t s = 0; s < h->n_seg; ++s) {
+    A.seg_first[s] = h->seg_first[s];
+    A.seg_start[s] = h->seg_start[s];
+    A.seg_len[s] = h->seg_len[s];
+  }
   // Adam's bias correction of the unrolled sums [MicroAdam ¶1]:
   // m_hat = (1-beta1)/(1-beta1^t) * sum_r beta1^r V_r, likewise v_hat.
   A.f1 = (float)((1.0 - b1) / (1.0 - std::pow(b1, (double)t)));
@@ -265,7 +323,8 @@ int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float l
 
 int mua_set_select_variant(mua_t h, int32_t variant) {
   if (!h || variant < 0 || variant > 2) return MUA_ERR_ARG;
-  if (variant == 2 && !((h->Bd % 32) == 0 && h->nb >= 2)) return MUA_ERR_UNSUPPORTED;
+  if (variant == 2 && !((h->Bd % 32) == 0 && h->nb >= 2 && h->n_seg == 0))
+    return MUA_ERR_UNSUPPORTED;
   // The CTA shapes hold the update's shared memory too (and variant 2 a copy
   // of the block): it must fit one CTA's 227 KB beside the static arrays.
   const uint32_t stage = variant == 2 ? ((2u * (uint32_t)h->Bd + (uint32_t)h->Bd / 2u + 127u) & ~127u) : 0u;

@@ -29,8 +29,9 @@ __global__ void __launch_bounds__(T, (T == 256 ? 5 : (T <= 512 ? 1024 / T : 1)))
   const int tid = threadIdx.x;
   const Geometry& G = A.g;
   const int j = G.nb - 1 - (int)blockIdx.x;
-  const int64_t start = (int64_t)j * G.Bd;
-  const int L = (j == G.nb - 1) ? G.last_len : G.Bd;
+  int64_t start;
+  int L;
+  block_span(A, j, start, L);
 
   load_weights(A, s_w1, s_w2);
 

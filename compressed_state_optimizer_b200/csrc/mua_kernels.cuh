@@ -26,6 +26,7 @@ constexpr int kElemsPerThread = 32;
 constexpr int kChunk = 8;
 constexpr int kChunks = kElemsPerThread / kChunk;
 constexpr int kMaxWindow = 64;            // m <= 64 (ages fit a 6-bit field)
+constexpr int kMaxSegments = 512;         // tensors of a list cut into blocks one by one
 constexpr int kMaxWindowEntries = 15360;  // m * row_stride per block, on chip
 constexpr int kCandCap = 2048;            // select: on-chip candidate list
 constexpr int kHistBins = 2048;           // radix digit of 11 bits
@@ -73,7 +74,34 @@ struct StepArgs {
   float w1[kMaxWindow];  // fp32(beta1^r), r = age
   float w2[kMaxWindow];  // fp32(beta2^r)
   uint32_t keys[10][2];  // Philox round keys: seed + r*(W0, W1)
+  // Tensor lists cut per tensor (n_seg > 0): segment s holds elements
+  // [seg_start[s], seg_start[s] + seg_len[s]) and blocks seg_first[s] ..
+  // seg_first[s+1]-1 (a ragged last block each). n_seg == 0: the flat cut.
+  int32_t n_seg;
+  int32_t seg_first[kMaxSegments];
+  int64_t seg_start[kMaxSegments];
+  int64_t seg_len[kMaxSegments];
 };
+
+// Start (element offset within the handle) and length of block j. Kernels
+// that call this take their StepArgs as a __grid_constant__ argument, so the
+// indexed reads stay in the parameter bank.
+__device__ __forceinline__ void block_span(const StepArgs& A, int j, int64_t& start, int& L) {
+  const Geometry& G = A.g;
+  if (A.n_seg == 0) {
+    start = (int64_t)j * G.Bd;
+    L = (j == G.nb - 1) ? G.last_len : G.Bd;
+    return;
+  }
+  int lo = 0, hi = A.n_seg - 1;  // the last segment whose first block is <= j
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (A.seg_first[mid] <= j) lo = mid; else hi = mid - 1;
+  }
+  const int64_t off = (int64_t)(j - A.seg_first[lo]) * G.Bd;
+  start = A.seg_start[lo] + off;
+  L = (int)min((int64_t)G.Bd, A.seg_len[lo] - off);
+}
 
 __device__ __forceinline__ bool update_in_select(const StepArgs& A, int j) {
   return (j & 7) < A.update_split;

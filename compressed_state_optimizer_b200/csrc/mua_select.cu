@@ -377,8 +377,9 @@ __device__ __forceinline__ void select_block(const StepArgs& A, int j,
   const int lane = tid & 31, wid = tid >> 5;
   constexpr int NW = T / 32;
   const Geometry& G = A.g;
-  const int64_t start = (int64_t)j * G.Bd;
-  const int L = (j == G.nb - 1) ? G.last_len : G.Bd;
+  int64_t start;
+  int L;
+  block_span(A, j, start, L);
   const int k = (int)(((int64_t)L * G.kb + G.Bd - 1) / G.Bd);
 
   for (int b = tid; b < kHistBins; b += T) hist[b] = 0u;  // used after later barriers
@@ -510,8 +511,9 @@ __global__ void __launch_bounds__(T, (T <= 512 ? 1024 / T : 1))
   extern __shared__ __align__(128) uint8_t dyn[];
   __shared__ SelectShared sh;
   const int j = blockIdx.x;
-  const int64_t start = (int64_t)j * A.g.Bd;
-  const int L = (j == A.g.nb - 1) ? A.g.last_len : A.g.Bd;
+  int64_t start;
+  int L;
+  block_span(A, j, start, L);
   uint4 gv[kChunks];
   uint32_t cv[kChunks];
   load_block<T, VEC>(A.grads, A.codes, start, L, threadIdx.x, gv, cv);

@@ -233,7 +233,8 @@ __device__ __forceinline__ void warp_radix(int hi, uint32_t prefix, int k, uint3
 }
 
 template <bool VEC, int MASKW>
-__global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const StepArgs A) {
+__global__ void __launch_bounds__(kWarps * 32, 3)
+    mua_select_warp_kernel(const __grid_constant__ StepArgs A) {
   extern __shared__ __align__(16) uint8_t dyn[];
   CtaSmem<MASKW>& S = *reinterpret_cast<CtaSmem<MASKW>*>(dyn);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -248,8 +249,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3) mua_select_warp_kernel(const S
   if (j >= G.nb) return;
   WarpSmem<MASKW>& W = S.w[wid];
   const float* lv = S.levels;
-  const int64_t start = (int64_t)j * G.Bd;
-  const int L = (j == G.nb - 1) ? G.last_len : G.Bd;
+  int64_t start;
+  int L;
+  block_span(A, j, start, L);
   const int k = (int)(((int64_t)L * G.kb + G.Bd - 1) / G.Bd);
   uint32_t* row = A.window + ((int64_t)j * G.m + A.row) * G.kp;
   const int nsteps = (L + 255) >> 8;

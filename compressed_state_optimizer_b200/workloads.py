@@ -66,6 +66,11 @@ class Workload:
     eps: float = 1e-8
     wd: float = 0.0
     seed: int = 0x5EED0000
+    per_tensor: bool = False       # blocks cut per tensor of ``shapes`` (else over the flat vector)
+
+    def segments(self):
+        """Tensor lengths when blocks are cut per tensor, else None."""
+        return [numel([s]) for s in self.shapes] if self.per_tensor else None
 
     def tensor_sizes(self) -> list[int]:
         if not self.shapes:

@@ -91,6 +91,26 @@ int mua_create_shard(int64_t d_total, int32_t block_size, int32_t k_per_block,
                      int32_t window, int32_t bits, int64_t block_begin,
                      int64_t block_count, mua_t* out);
 
+/*
+ * mua_create_segmented — like mua_create for a tensor list: the d-vector is
+ * the concatenation of n_seg tensors of lengths seg_len[0..n_seg) (d is their
+ * sum, elements in list order), and each tensor is cut into its own blocks of
+ * B_d, the last one ragged (k = ceil(L * k_b / B_d) entries), so no block spans
+ * two tensors. delta and Delta stay global over the d-vector [MicroAdam ¶1].
+ * Blocks are numbered tensor by tensor; the state layout, window rows and
+ * random draws (by global element index) are those of the flat case with that
+ * block count. seg_len is read during the call only. Host only.
+ * Errors: MUA_ERR_ARG for NULL pointers, n_seg < 1, a length < 1 or the
+ * arguments mua_create rejects; MUA_ERR_UNSUPPORTED for an odd length (a
+ * block must start on a byte of the 4-bit codes), n_seg > MUA_MAX_SEGMENTS,
+ * and what mua_create cannot hold. Variant 2 of mua_set_select_variant is not
+ * available for these handles. The 16-byte vector path is used when B_d and
+ * every length are multiples of 8.
+ */
+#define MUA_MAX_SEGMENTS 512
+int mua_create_segmented(const int64_t* seg_len, int32_t n_seg, int32_t block_size,
+                         int32_t k_per_block, int32_t window, int32_t bits, mua_t* out);
+
 /* mua_destroy — release a handle (NULL is ignored). Host only. */
 void mua_destroy(mua_t h);
 
@@ -183,8 +203,8 @@ int mua_set_update_split(mua_t h, int32_t split);
  *     parameter updates then run in mua_apply (mua_set_update_split ignored);
  *   1 one CTA per block;
  *   2 persistent CTAs streaming each next block into shared memory with
- *     bulk copies (needs B_d % 32 == 0 and at least 2 blocks, else
- *     MUA_ERR_UNSUPPORTED).
+ *     bulk copies (needs B_d % 32 == 0, at least 2 blocks and a flat cut,
+ *     else MUA_ERR_UNSUPPORTED).
  * Variants 1 and 2 also return MUA_ERR_UNSUPPORTED when one block's select
  * and AdamStats working set does not fit one CTA's shared memory.
  * Host only; MUA_ERR_ARG for other values.

@@ -156,3 +156,43 @@ def test_shard_geometry(mua):
     assert a.layout.blocks + b.layout.blocks == whole.layout.blocks
     with pytest.raises(mua.MuaError):
         mua.MicroAdam(d, block_size=Bd, k_per_block=2, window=3, shard=(6, 6))
+
+
+def _create_seg(mua, segs, Bd=256, kb=3, m=5, bits=4):
+    import ctypes
+    lib = mua.library()
+    h = ctypes.c_void_p()
+    arr = (ctypes.c_int64 * max(1, len(segs)))(*segs)
+    rc = lib.mua_create_segmented(arr, len(segs), Bd, kb, m, bits, ctypes.byref(h))
+    return rc, h
+
+
+@pytest.mark.parametrize("segs,code", [
+    ([], -1),                       # no tensor
+    ([100, 0, 40], -1),             # empty tensor
+    ([100, 37, 40], -2),            # odd length: a block would start inside a code byte
+    ([2] * 513, -2),                # more than MUA_MAX_SEGMENTS
+])
+def test_create_segmented_rejects(mua, segs, code):
+    rc, h = _create_seg(mua, segs)
+    assert rc == code and not h.value
+
+
+def test_segmented_layout(mua):
+    """Blocks are counted tensor by tensor; the state is the flat layout of d with
+    that block count."""
+    segs = [1000, 256, 10, 512 + 2]
+    m = mua.MicroAdam(sum(segs), block_size=256, k_per_block=3, window=5, segments=segs)
+    nb = 4 + 1 + 1 + 3
+    d = sum(segs)
+    assert m.layout.blocks == nb == m.blocks and m.d == d
+    codes_bytes = -(-((d + 1) // 2) // 256) * 256
+    assert m.layout.window == 256 + codes_bytes
+    assert m.state_bytes == 256 + codes_bytes + 4 * nb * 5 * 4 == m.layout.bytes
+    with pytest.raises(ValueError):
+        mua.MicroAdam(d + 2, block_size=256, k_per_block=3, window=5, segments=segs)
+    # the persistent select shape needs the flat cut
+    with pytest.raises(mua.MuaError):
+        m.set_select_variant(2)
+    m.set_select_variant(1)
+    m.set_select_variant(0)

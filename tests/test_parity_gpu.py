@@ -63,18 +63,18 @@ def compare_stats(mhat, vhat, stats, what=""):
 
 def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0.9,
                b2=0.999, eps=1e-8, wd=0.0, grads_fn=None, stats=True, use_step=False,
-               split=None, variant=None):
+               split=None, variant=None, segments=None):
     torch, MicroAdam, workloads = _mods()
     w = workloads.Workload("parity", d, Bd, kb, m, kind, steps, seed=seed)
     p0 = workloads.make_params(d, seed=7)
-    mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m)
+    mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m, segments=segments)
     if variant is not None:
         mo.set_select_variant(variant)
     if split is not None:
         mo.set_update_split(split)
     state = mo.new_state("cuda")
     p_gpu = p0.cuda()
-    ost = oracle.new_state(d, Bd, kb, m)
+    ost = oracle.new_state(d, Bd, kb, m, segments=segments)
     p_ref = p0.numpy().copy()
     hyper = dict(lr=lr, beta1=b1, beta2=b2, eps=eps, wd=wd)
     for t in range(1, steps + 1):
@@ -238,3 +238,24 @@ def _structured_grads(d, Bd, seed):
 def test_select_paths(kb):
     d, Bd = 8 * 16384 + 999, 16384
     run_parity(d, Bd, kb, 3, 4, grads_fn=_structured_grads(d, Bd, 99 + kb))
+
+
+SEGMENTED = [
+    # (B_d, k_b, m, steps, tensor lengths, kind, select variant)
+    (16384, 164, 4, 8, [2 * 16384 + 1000, 8000, 16384, 4096 + 8, 30000], "t3", None),
+    (16384, 164, 4, 6, [2 * 16384 + 1000, 8000, 16384, 4096 + 8, 30000], "t3", 1),
+    (2048, 21, 3, 6, [5000, 2, 2048, 3070, 6], "normal", None),  # lengths not all 8k: scalar path
+    (8192, 82, 10, 12, [8192 * 3, 4104, 9000, 1000], "t3", None),
+]
+
+
+@pytest.mark.parametrize("Bd,kb,m,steps,segs,kind,variant", SEGMENTED)
+def test_segmented(Bd, kb, m, steps, segs, kind, variant):
+    """A tensor list cut per tensor (each tensor's last block ragged) against the
+    oracle's per-tensor cut."""
+    run_parity(sum(segs), Bd, kb, m, steps, kind=kind, segments=segs, variant=variant)
+
+
+def test_segmented_step():
+    segs = [3 * 4096 + 64, 512, 4096]
+    run_parity(sum(segs), 4096, 41, 5, 8, kind="t3", segments=segs, use_step=True, wd=0.05)
