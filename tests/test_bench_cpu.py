@@ -1,0 +1,36 @@
+"""bench.py's reference arm (the CPU oracle timed on a bounded sample) runs
+without a GPU and prints one JSON line with the fields of the benchmark
+contract."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_reference_arm_json_line(oracle_lib):
+    out = subprocess.run(
+        [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+         "flat_1m", "--steps", "2", "--warmup", "1", "--cpu-sample", "32768"],
+        capture_output=True, text=True, timeout=300, cwd=ROOT, check=True).stdout
+    lines = [ln for ln in out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "Gparams/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["steps"] == 2 and d["warmup"] == 1
+    assert d["n_gpus"] == 1 and d["config"]["workload"] == "flat_d2^20_normal"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_workload_names():
+    sys.path.insert(0, ROOT)
+    import bench
+    for name, d in [("llama2_7b", 6738415616), ("llama2_7b_per_tensor", 6738415616),
+                    ("flat_134m", 1 << 27), ("bert_base_2048", 108888576),
+                    ("flat_1g_m37", 1 << 30)]:
+        assert bench.get_workload(name).d == d
+    w = bench.get_workload("llama2_7b_per_tensor", wd=0.1)
+    assert w.wd == 0.1 and len(w.segments()) == 291 and sum(w.segments()) == w.d
+    assert bench.get_workload("llama2_7b").segments() is None
