@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama2_7b",
                     help="llama2_7b | llama2_7b_per_tensor | flat_134m | flat_1m | bert_base | "
-                         "bert_base_<B_d> | flat_1g_m<m>")
+                         "bert_base_<B_d>[_per_tensor] | flat_1g_m<m>")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--update-split", type=int, default=None,
@@ -78,9 +78,13 @@ def _named_workload(name):
         return W.flat_small()
     if name == "bert_base":
         return W.bert_base()
-    m = re.fullmatch(r"bert_base_(\d+)", name)
+    m = re.fullmatch(r"bert_base_(\d+)(_per_tensor)?", name)
     if m:
-        return W.bert_base(int(m.group(1)))
+        w = W.bert_base(int(m.group(1)))
+        if m.group(2):
+            import dataclasses
+            w = dataclasses.replace(w, name=w.name + "_per_tensor", per_tensor=True)
+        return w
     m = re.fullmatch(r"flat_1g_m(\d+)", name)
     if m:
         return W.flat_1g(int(m.group(1)))
