@@ -392,7 +392,7 @@ def run_ours(args, rank, world, local_rank):
         }
         if e2e is not None:
             line["e2e"] = e2e
-        if not args.no_cpu_baseline:
+        if not args.no_cpu_baseline and world == 1:  # the oracle's timing: rank 0 at N = 1 only
             line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
         print(json.dumps(line), flush=True)
 
