@@ -72,6 +72,24 @@ int pick_threads(int Bd) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Warps of the apply kernel resident per SM at CTA size T: limited by its
+// launch bound (5 CTAs of 256, else 1024 / T CTAs), by shared memory (228 KB
+// per SM, 1 KB reserved per CTA) and by 2048 threads.
+int apply_warps_per_sm(int T, int Bd, int kp, int m) {
+  const int by_bound = T == 256 ? 5 : (T <= 512 ? 1024 / T : 1);
+  const int by_smem = (228 * 1024) / ((int)mua::apply_smem_bytes(T, Bd, kp, m) + 1024);
+  const int by_threads = 2048 / T;
+  return std::min(by_bound, std::min(by_smem, by_threads)) * (T / 32);
+}
+
+// Half the select CTA (the block in two passes; more CTAs per SM, so one
+// CTA's update barriers overlap the others' codec) unless the update's
+// shared memory makes the full CTA keep more warps resident (long windows).
+int pick_apply_threads(int T, int Bd, int kp, int m) {
+  if (T < 64) return T;
+  return apply_warps_per_sm(T / 2, Bd, kp, m) >= apply_warps_per_sm(T, Bd, kp, m) ? T / 2 : T;
+}
+
 int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
          int64_t block_begin, int64_t block_count, mua_t* out) {
   if (!out) return MUA_ERR_ARG;
@@ -101,7 +119,7 @@ int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
   h->m = m;
   h->last_len = (int32_t)(h->d - (block_count - 1) * Bd);
   h->threads = pick_threads(Bd);
-  h->apply_threads = h->threads >= 64 ? h->threads / 2 : h->threads;
+  h->apply_threads = pick_apply_threads(h->threads, Bd, kp, m);
   h->vec = (Bd % 8) == 0;
   h->persistent = false;
   h->variant = 0;
