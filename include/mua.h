@@ -190,6 +190,8 @@ int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float 
 /*
  * mua_set_update_split — which kernel applies stage (6) to block j: mua_select
  * when (j mod 8) < split, mua_apply otherwise; 0 <= split <= 8 (default 4).
+ * Only the CTA shapes of mua_select (variants 1, 2) use it: with the default
+ * warp-per-block select every block is updated in mua_apply.
  * The results do not depend on it (each block is updated exactly once, by
  * the same arithmetic); it only moves HBM traffic between the two kernels to
  * balance them. Host only; MUA_ERR_ARG when out of range.
