@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.mua_oracle_bf16_to_f32.restype = f32
         L.mua_oracle_f32_to_bf16.argtypes = [f32]
         L.mua_oracle_f32_to_bf16.restype = ctypes.c_uint16
+        L.mua_oracle_f64_to_bf16.argtypes = [f64]
+        L.mua_oracle_f64_to_bf16.restype = ctypes.c_uint16
         L.mua_oracle_dequantize.argtypes = [P, i64, f32, f32, P]
         L.mua_oracle_dequantize.restype = None
         L.mua_oracle_quantize.argtypes = [P, i64, i64, f32, f32, i64, u64, P]
@@ -69,6 +71,9 @@ def lib() -> ctypes.CDLL:
         L.mua_oracle_step_seg.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P,
                                           f64, f64, f64, f64, f64, i64, u64, P, P, P]
         L.mua_oracle_step_seg.restype = ctypes.c_int
+        L.mua_oracle_step_seg_bf16.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P, P,
+                                               f64, f64, f64, f64, f64, i64, u64, P, P, P]
+        L.mua_oracle_step_seg_bf16.restype = ctypes.c_int
         L.mua_oracle_num_blocks.argtypes = [P, i32, i32]
         L.mua_oracle_num_blocks.restype = i64
         _lib = L
@@ -103,6 +108,11 @@ def bf16_to_f32(h: int) -> float:
 
 def f32_to_bf16(x: float) -> int:
     return int(lib().mua_oracle_f32_to_bf16(x))
+
+
+def f64_to_bf16(x: float) -> int:
+    """bf16 bits of an fp64 value rounded once, to nearest with ties to even."""
+    return int(lib().mua_oracle_f64_to_bf16(x))
 
 
 def block_k(L: int, Bd: int, kb: int) -> int:
@@ -184,31 +194,40 @@ def new_state(d: int, Bd: int, kb: int, m: int, segments=None) -> OracleState:
 
 def step(st: OracleState, p: np.ndarray, g_bits: np.ndarray, *, lr: float, beta1: float,
          beta2: float, eps: float, wd: float, t: int, seed: int,
-         want_stats: bool = False):
-    """One MicroAdam step in place on ``st`` and ``p`` (float32[d]).
+         want_stats: bool = False, p_exact: np.ndarray | None = None):
+    """One MicroAdam step in place on ``st`` and ``p``.
 
-    ``g_bits`` is the bf16 gradient as uint16 bits. The fp32 hyper-parameters
-    are widened exactly to fp64. Returns ``(m_hat, v_hat, m_abs)`` as fp64
-    arrays when ``want_stats`` is set, else None.
+    ``p`` holds the parameters: float32[d], or uint16[d] bf16 bits (each changed
+    parameter is then rounded once to bf16; ``p_exact``, float64[d], receives
+    the values before that rounding). ``g_bits`` is the bf16 gradient as
+    uint16 bits. The fp32 hyper-parameters are widened exactly to fp64.
+    Returns ``(m_hat, v_hat, m_abs)`` as fp64 arrays when ``want_stats`` is
+    set, else None.
     """
-    assert p.dtype == np.float32 and p.size == st.d and p.flags["C_CONTIGUOUS"]
+    assert p.dtype in (np.float32, np.uint16) and p.size == st.d and p.flags["C_CONTIGUOUS"]
     g_bits = np.ascontiguousarray(g_bits, dtype=np.uint16)
     assert g_bits.size == st.d
     stats = None
     if want_stats:
         stats = tuple(np.zeros(st.d, dtype=np.float64) for _ in range(3))
     f = lambda v: float(np.float32(v))  # noqa: E731  (the fp32 value the kernels see)
-    if st.segs is None:
+    segs = st.segs if st.segs is not None else np.array([st.d], dtype=np.int64)
+    tail = (f(lr), f(beta1), f(beta2), f(eps), f(wd), t, seed,
+            *(_ptr(s) for s in (stats or (None,) * 3)))
+    if p.dtype == np.uint16:
+        if p_exact is not None:
+            assert p_exact.dtype == np.float64 and p_exact.size == st.d
+        rc = lib().mua_oracle_step_seg_bf16(_ptr(segs), segs.size, st.Bd, st.kb, st.m, _ptr(p),
+                                            _ptr(p_exact), _ptr(g_bits), _ptr(st.codes),
+                                            _ptr(st.scal), _ptr(st.G_idx), _ptr(st.G_val), *tail)
+    elif st.segs is None:
         rc = lib().mua_oracle_step(st.d, st.Bd, st.kb, st.m, _ptr(p), _ptr(g_bits),
                                    _ptr(st.codes), _ptr(st.scal), _ptr(st.G_idx),
-                                   _ptr(st.G_val), f(lr), f(beta1), f(beta2), f(eps), f(wd),
-                                   t, seed, *(_ptr(s) for s in (stats or (None,) * 3)))
+                                   _ptr(st.G_val), *tail)
     else:
         rc = lib().mua_oracle_step_seg(_ptr(st.segs), st.segs.size, st.Bd, st.kb, st.m,
                                        _ptr(p), _ptr(g_bits), _ptr(st.codes), _ptr(st.scal),
-                                       _ptr(st.G_idx), _ptr(st.G_val), f(lr), f(beta1),
-                                       f(beta2), f(eps), f(wd), t, seed,
-                                       *(_ptr(s) for s in (stats or (None,) * 3)))
+                                       _ptr(st.G_idx), _ptr(st.G_val), *tail)
     if rc != 0:
         raise ValueError("oracle step rejected its arguments")
     return stats

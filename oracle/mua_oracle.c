@@ -33,6 +33,9 @@
  *    with beta2 and V^2 (Adam's bias-corrected moments), r = age of the row.
  *  - update u = m_hat / (eps + sqrt(v_hat)); decoupled weight decay
  *    p <- p*(1 - lr*wd) is applied to every coordinate before the update.
+ *  - bf16 parameters (no fp32 copy, the page's 7B fine-tune on one 40 GB
+ *    GPU): every parameter the step changes is rounded once to bf16, to
+ *    nearest with ties to even.
  *  - delta, Delta are global over the flat d-vector; blocks are cut over
  *    that vector, or, for a tensor list, over each tensor (segment) in turn;
  *    a ragged last block of length L keeps k = ceil(L*k_b/B_d) entries.
@@ -102,6 +105,28 @@ uint16_t mua_oracle_f32_to_bf16(float f) {
         return (uint16_t)((b >> 16) | 0x0040u);
     uint32_t lsb = (b >> 16) & 1u;
     return (uint16_t)((b + 0x7FFFu + lsb) >> 16);
+}
+
+/* Round an fp64 value to bf16 (8 significant bits, the binary32 exponent
+ * range) to nearest, ties to even, in one rounding: the value is scaled by a
+ * power of two so that its bf16 unit in the last place becomes 1, rounded to
+ * an integer with ties to even, and scaled back (all exact in fp64). Values
+ * past the largest bf16 become +-inf; NaN stays NaN. */
+uint16_t mua_oracle_f64_to_bf16(double x) {
+    if (isnan(x)) return (uint16_t)0x7FC0u;
+    if (x == 0.0) return (uint16_t)(signbit(x) ? 0x8000u : 0x0000u);
+    int e;
+    frexp(x, &e);                      /* |x| = f * 2^e, 0.5 <= f < 1 */
+    int q = e - 1;                     /* floor(log2 |x|) */
+    if (q < -126) q = -126;            /* subnormal bf16 share the spacing 2^-133 */
+    const double ulp = ldexp(1.0, q - 7);
+    double y = x / ulp;                /* exact: a power-of-two scaling */
+    double r = floor(y);
+    const double frac = y - r;         /* exact */
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    r = copysign(r * ulp, x);          /* a value that rounds to zero keeps its sign */
+    if (fabs(r) >= ldexp(1.0, 128)) return (uint16_t)(r > 0 ? 0x7F80u : 0xFF80u);
+    return (uint16_t)(bits_from_f32((float)r) >> 16);   /* r is a bf16 value: exact */
 }
 
 /* ---------------------------------------------------------------------- */
@@ -199,12 +224,18 @@ int64_t mua_oracle_num_blocks(const int64_t* seg, int32_t n_seg, int32_t Bd) {
 }
 
 /* One MicroAdam step [MicroAdam ¶1] over the concatenation of n_seg segments
- * of lengths seg[0..n_seg) (d = their sum), blocks cut per segment. */
-int mua_oracle_step_seg(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, int32_t m,
-                        float* p, const uint16_t* g, uint8_t* codes, float* scal,
-                        int16_t* G_idx, uint16_t* G_val, double lr, double beta1,
-                        double beta2, double eps, double wd, int64_t t, uint64_t seed,
-                        double* mhat, double* vhat, double* mabs) {
+ * of lengths seg[0..n_seg) (d = their sum), blocks cut per segment. The
+ * parameters are fp32 (p32) or, when p16 is given instead, bf16 bits: then
+ * each parameter the step changes is computed in fp64 from its bf16 value and
+ * rounded once to bf16, nearest-even (there is no fp32 copy); p_exact, if
+ * given, receives that fp64 value before the rounding (and f32(p) for the
+ * parameters the step leaves alone). */
+static int step_impl(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, int32_t m,
+                     float* p32, uint16_t* p16, double* p_exact, const uint16_t* g,
+                     uint8_t* codes, float* scal, int16_t* G_idx, uint16_t* G_val, double lr,
+                     double beta1, double beta2, double eps, double wd, int64_t t,
+                     uint64_t seed, double* mhat, double* vhat, double* mabs) {
+    if ((p32 == NULL) == (p16 == NULL)) return -1;
     if (n_seg < 1 || Bd < 1 || Bd > 32766 || kb < 1 || kb > Bd || m < 1 || t < 1) return -1;
     int64_t d = 0;
     for (int32_t s = 0; s < n_seg; ++s) {
@@ -323,15 +354,41 @@ int mua_oracle_step_seg(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t k
         if (mhat) mhat[q] = m_hat;
         if (vhat) vhat[q] = v_hat;
         if (mabs) mabs[q] = f1 * za[q];
-        double pq = (double)p[q];
+        double pq = p32 ? (double)p32[q] : (double)mua_oracle_bf16_to_f32(p16[q]);
         if (wd != 0.0) pq = pq * decay;
         if (touched[q]) pq = pq - lr * (m_hat / (eps + sqrt(v_hat)));
-        if (wd != 0.0 || touched[q]) p[q] = (float)pq;
+        if (p_exact) p_exact[q] = pq;
+        if (wd != 0.0 || touched[q]) {
+            if (p32) p32[q] = (float)pq;
+            else p16[q] = mua_oracle_f64_to_bf16(pq);
+        }
     }
 
     free(a); free(order); free(z1); free(z2); free(za); free(touched);
     free(bstart); free(blen);
     return 0;
+}
+
+int mua_oracle_step_seg(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, int32_t m,
+                        float* p, const uint16_t* g, uint8_t* codes, float* scal,
+                        int16_t* G_idx, uint16_t* G_val, double lr, double beta1,
+                        double beta2, double eps, double wd, int64_t t, uint64_t seed,
+                        double* mhat, double* vhat, double* mabs) {
+    if (p == NULL) return -1;
+    return step_impl(seg, n_seg, Bd, kb, m, p, NULL, NULL, g, codes, scal, G_idx, G_val, lr,
+                     beta1, beta2, eps, wd, t, seed, mhat, vhat, mabs);
+}
+
+/* The same step with bf16 parameters (see step_impl). */
+int mua_oracle_step_seg_bf16(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb,
+                             int32_t m, uint16_t* p16, double* p_exact, const uint16_t* g,
+                             uint8_t* codes, float* scal, int16_t* G_idx, uint16_t* G_val,
+                             double lr, double beta1, double beta2, double eps, double wd,
+                             int64_t t, uint64_t seed, double* mhat, double* vhat,
+                             double* mabs) {
+    if (p16 == NULL) return -1;
+    return step_impl(seg, n_seg, Bd, kb, m, NULL, p16, p_exact, g, codes, scal, G_idx, G_val,
+                     lr, beta1, beta2, eps, wd, t, seed, mhat, vhat, mabs);
 }
 
 /* The flat cut: one segment of length d. */

@@ -347,6 +347,108 @@ def check_reduces_to_adam(wd: float = 0.0):
         np.testing.assert_allclose(p, ref[t - 1], rtol=2e-6, atol=2e-6 * lr)
 
 
+# --------------------------------------------------------------- bf16 parameters
+def _bf16_table():
+    """Every finite bf16 value (exact, as float64) with its bit pattern, sorted."""
+    bits = np.arange(1 << 16, dtype=np.uint32)
+    with np.errstate(invalid="ignore"):  # the NaN patterns, dropped below
+        vals = (bits << 16).astype(np.uint32).view(np.float32).astype(np.float64)
+    keep = np.isfinite(vals)
+    vals, bits = vals[keep], bits[keep].astype(np.uint16)
+    order = np.argsort(vals, kind="stable")
+    vals, bits = vals[order], bits[order]
+    # -0 and +0 compare equal: keep +0 only for the neighbour search
+    keep = ~((vals == 0) & (bits == 0x8000))
+    return vals[keep], bits[keep]
+
+
+def _nearest_bf16(x: float, vals, bits) -> int:
+    """Nearest bf16 of x by search over the whole bf16 set: the two values that
+    bracket x, the nearer one in exact rational arithmetic, a tie to the even
+    bit pattern."""
+    from fractions import Fraction
+    if x == 0.0:
+        return 0x8000 if np.signbit(x) else 0
+    i = int(np.searchsorted(vals, x))
+    cands = [j for j in (i - 1, i) if 0 <= j < vals.size]
+    fx = Fraction(x)
+    dist = [abs(Fraction(float(vals[j])) - fx) for j in cands]
+    best = min(dist)
+    pick = [cands[k] for k in range(len(cands)) if dist[k] == best]
+    if len(pick) == 2:
+        pick = [j for j in pick if (int(bits[j]) & 1) == 0]
+    b = int(bits[pick[0]])
+    if float(vals[pick[0]]) == 0.0 and x < 0:
+        b = 0x8000
+    return b
+
+
+def check_f64_to_bf16_rne():
+    """The oracle's one-step fp64 -> bf16 rounding equals the nearest bf16 found
+    by search over all bf16 values (ties to even), on random values across
+    magnitudes, exact midpoints, and the subnormal range."""
+    vals, bits = _bf16_table()
+    rng = np.random.default_rng(77)
+    xs = list(rng.standard_normal(300) * 10.0 ** rng.integers(-30, 30, 300))
+    xs += list(rng.standard_normal(100) * 1e-39)               # subnormal bf16 range
+    b16 = rng.integers(0x0080, 0x7F00, 200).astype(np.uint32)  # midpoints of neighbours
+    lo = (b16 << 16).view(np.float32).astype(np.float64)
+    hi = ((b16 + 1) << 16).view(np.float32).astype(np.float64)
+    xs += list((lo + hi) / 2) + list(-(lo + hi) / 2)
+    xs += list(np.nextafter((lo + hi) / 2, np.inf)) + list(np.nextafter((lo + hi) / 2, -np.inf))
+    for x in xs:
+        assert oracle.f64_to_bf16(float(x)) == _nearest_bf16(float(x), vals, bits), x
+
+
+def _bf16_midpoint_distance(x: np.ndarray) -> np.ndarray:
+    """Relative distance of each fp64 value to the nearest midpoint between two
+    neighbouring bf16 values (where a rounding decision can flip)."""
+    f = x.astype(np.float32)
+    b = (f.view(np.uint32) >> 16).astype(np.uint32)
+    lo = (b << 16).view(np.float32).astype(np.float64)
+    hi = ((b + 1) << 16).view(np.float32).astype(np.float64)
+    mid = (lo + hi) / 2
+    return np.abs(x - mid) / np.maximum(np.abs(x), 1e-30)
+
+
+def check_bf16_params_reduce_to_adam(wd: float = 0.0):
+    """bf16 parameters: with k_b = B_d and m >= T the step is Adam (AdamW when
+    wd > 0) on the bf16 gradients with the parameter stored back in bf16 after
+    every step. Reference: torch.optim on an fp32 copy of the bf16 parameter
+    each step, stored with torch's own bf16 conversion. The two may disagree by
+    one bf16 step only where the exact value sits within 1e-5 of a rounding
+    midpoint (torch rounds an fp32 intermediate)."""
+    Bd = 250
+    d, T = 4 * Bd, 8
+    lr, b1, b2, eps = 1e-2, 0.9, 0.999, 1e-8
+    p0 = torch.from_numpy((np.random.default_rng(18).standard_normal(d) * 0.02)
+                          .astype(np.float32)).to(torch.bfloat16)
+    grads = [normal_bf16(d, 900 + t) for t in range(1, T + 1)]
+    q = torch.zeros(d, dtype=torch.float32, requires_grad=True)
+    opt = (torch.optim.AdamW([q], lr=lr, betas=(b1, b2), eps=eps, weight_decay=wd) if wd
+           else torch.optim.Adam([q], lr=lr, betas=(b1, b2), eps=eps))
+    p_ref = p0.clone()
+    st = oracle.new_state(d, Bd, Bd, T)
+    p = p0.view(torch.int16).numpy().view(np.uint16).copy()
+    exact = np.zeros(d, dtype=np.float64)
+    moved = 0
+    for t in range(1, T + 1):
+        with torch.no_grad():
+            q.copy_(p_ref.float())
+        q.grad = torch.from_numpy(f32_of_bits(grads[t - 1]).copy())
+        opt.step()
+        p_ref = q.detach().to(torch.bfloat16)
+        want = p_ref.view(torch.int16).numpy().view(np.uint16)
+        oracle.step(st, p, grads[t - 1], lr=lr, beta1=b1, beta2=b2, eps=eps, wd=wd, t=t,
+                    seed=3, p_exact=exact)
+        diff = np.flatnonzero(p != want)
+        assert np.all(_bf16_midpoint_distance(exact[diff]) < 1e-5), (t, diff[:5])
+        assert diff.size <= 2
+        moved += int(np.count_nonzero(p != p0.view(torch.int16).numpy().view(np.uint16)))
+        p_ref = torch.from_numpy(p.view(np.int16).copy()).view(torch.bfloat16)  # resync
+    assert moved > 0
+
+
 # --------------------------------------------------------------- Lemma 3 / sparsity
 def check_lemma3_bound(Bd: int = 8, kb: int = 4, steps: int = 200, seeds: int = 64):
     """[MicroAdam ¶3, Lemma 3] ||e_t||^2 <= 4 q_w^2 G^2 / (1 - q_w^2)^2 on tiny runs,
@@ -489,6 +591,8 @@ ALL = [check_philox_vs_torch, check_draw16_mapping, check_draw16_uniform, check_
        check_quant_exact_levels, check_quant_error_bound, check_quant_unbiased,
        check_lemma1_per_realization, check_adamstats_vs_dense_ema, check_closed_form_m1_t1,
        check_reduces_to_adam, functools.partial(check_reduces_to_adam, wd=0.1),
+       check_f64_to_bf16_rne, check_bf16_params_reduce_to_adam,
+       functools.partial(check_bf16_params_reduce_to_adam, wd=0.1),
        check_lemma3_bound, check_update_sparsity, check_block_locality,
        check_segmented_topk_minmax_step1, check_segmented_update_support,
        check_segmented_whole_blocks_equal_flat]

@@ -79,6 +79,15 @@ MUTANTS = {
     "weight_decay_dropped": (
         "if (wd != 0.0) pq = pq * decay;",
         ";"),
+    "bf16_params_truncated": (
+        "if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;",
+        ";"),
+    "bf16_params_ties_away_from_zero": (
+        "if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;",
+        "if (frac >= 0.5) r += 1.0;"),
+    "bf16_params_widened_as_integers": (
+        "double pq = p32 ? (double)p32[q] : (double)mua_oracle_bf16_to_f32(p16[q]);",
+        "double pq = p32 ? (double)p32[q] : (double)p16[q];"),
     "segment_cut_ignored": (
         "blen[j] = (seg[s] - b < Bd) ? (seg[s] - b) : Bd;",
         "blen[j] = (d - (off + b) < Bd) ? (d - (off + b)) : Bd;"),
