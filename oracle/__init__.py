@@ -24,60 +24,86 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "mua_oracle.c")
 _LIB = os.path.join(_HERE, "libmua_oracle.so")
+_LIB_OMP = os.path.join(_HERE, "libmua_oracle_omp.so")  # the same source with -fopenmp
 
 # gcc flags: IEEE fp32 with every operation rounded, no contraction into FMA.
 CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
 
+def _compile(out: str, extra, force: bool):
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(_SRC):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *CFLAGS, *extra, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, out)
+    return out
+
+
 def build(force: bool = False) -> str:
-    """Compile ``mua_oracle.c`` into ``libmua_oracle.so`` (next to it)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        tmp = _LIB + f".tmp{os.getpid()}"
-        subprocess.run(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"], check=True)
-        os.replace(tmp, _LIB)
-    return _LIB
+    """Compile ``mua_oracle.c`` into ``libmua_oracle.so`` and, with OpenMP over
+    blocks, ``libmua_oracle_omp.so`` (both next to it)."""
+    _compile(_LIB_OMP, ["-fopenmp"], force)
+    return _compile(_LIB, [], force)
 
 
 _lib = None
+_lib_omp = None
+
+
+def lib_openmp() -> ctypes.CDLL:
+    """The OpenMP build (bit-identical results; threads from OMP_NUM_THREADS or
+    ``set_threads``)."""
+    global _lib_omp
+    if _lib_omp is None:
+        _compile(_LIB_OMP, ["-fopenmp"], False)
+        _lib_omp = _declare(ctypes.CDLL(_LIB_OMP))
+    return _lib_omp
+
+
+def set_threads(n: int):
+    """Threads of the OpenMP build."""
+    lib_openmp().omp_set_num_threads(int(n))
 
 
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
         build()
-        L = ctypes.CDLL(_LIB)
-        P = ctypes.c_void_p
-        i64, i32, u64, f32, f64 = (ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64,
-                                   ctypes.c_float, ctypes.c_double)
-        L.mua_oracle_philox4x32_10.argtypes = [P, P, P]
-        L.mua_oracle_philox4x32_10.restype = None
-        L.mua_oracle_draw16.argtypes = [u64, i64, i64]
-        L.mua_oracle_draw16.restype = ctypes.c_uint32
-        L.mua_oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
-        L.mua_oracle_bf16_to_f32.restype = f32
-        L.mua_oracle_f32_to_bf16.argtypes = [f32]
-        L.mua_oracle_f32_to_bf16.restype = ctypes.c_uint16
-        L.mua_oracle_f64_to_bf16.argtypes = [f64]
-        L.mua_oracle_f64_to_bf16.restype = ctypes.c_uint16
-        L.mua_oracle_dequantize.argtypes = [P, i64, f32, f32, P]
-        L.mua_oracle_dequantize.restype = None
-        L.mua_oracle_quantize.argtypes = [P, i64, i64, f32, f32, i64, u64, P]
-        L.mua_oracle_quantize.restype = None
-        L.mua_oracle_block_k.argtypes = [i64, i32, i32]
-        L.mua_oracle_block_k.restype = i64
-        L.mua_oracle_step.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P,
-                                      f64, f64, f64, f64, f64, i64, u64, P, P, P]
-        L.mua_oracle_step.restype = ctypes.c_int
-        L.mua_oracle_step_seg.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P,
-                                          f64, f64, f64, f64, f64, i64, u64, P, P, P]
-        L.mua_oracle_step_seg.restype = ctypes.c_int
-        L.mua_oracle_step_seg_bf16.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P, P,
-                                               f64, f64, f64, f64, f64, i64, u64, P, P, P]
-        L.mua_oracle_step_seg_bf16.restype = ctypes.c_int
-        L.mua_oracle_num_blocks.argtypes = [P, i32, i32]
-        L.mua_oracle_num_blocks.restype = i64
-        _lib = L
+        _lib = _declare(ctypes.CDLL(_LIB))
     return _lib
+
+
+def _declare(L: ctypes.CDLL) -> ctypes.CDLL:
+    P = ctypes.c_void_p
+    i64, i32, u64, f32, f64 = (ctypes.c_int64, ctypes.c_int32, ctypes.c_uint64,
+                               ctypes.c_float, ctypes.c_double)
+    L.mua_oracle_philox4x32_10.argtypes = [P, P, P]
+    L.mua_oracle_philox4x32_10.restype = None
+    L.mua_oracle_draw16.argtypes = [u64, i64, i64]
+    L.mua_oracle_draw16.restype = ctypes.c_uint32
+    L.mua_oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+    L.mua_oracle_bf16_to_f32.restype = f32
+    L.mua_oracle_f32_to_bf16.argtypes = [f32]
+    L.mua_oracle_f32_to_bf16.restype = ctypes.c_uint16
+    L.mua_oracle_f64_to_bf16.argtypes = [f64]
+    L.mua_oracle_f64_to_bf16.restype = ctypes.c_uint16
+    L.mua_oracle_dequantize.argtypes = [P, i64, f32, f32, P]
+    L.mua_oracle_dequantize.restype = None
+    L.mua_oracle_quantize.argtypes = [P, i64, i64, f32, f32, i64, u64, P]
+    L.mua_oracle_quantize.restype = None
+    L.mua_oracle_block_k.argtypes = [i64, i32, i32]
+    L.mua_oracle_block_k.restype = i64
+    L.mua_oracle_step.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P,
+                                  f64, f64, f64, f64, f64, i64, u64, P, P, P]
+    L.mua_oracle_step.restype = ctypes.c_int
+    L.mua_oracle_step_seg.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P,
+                                      f64, f64, f64, f64, f64, i64, u64, P, P, P]
+    L.mua_oracle_step_seg.restype = ctypes.c_int
+    L.mua_oracle_step_seg_bf16.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, P, P,
+                                           f64, f64, f64, f64, f64, i64, u64, P, P, P]
+    L.mua_oracle_step_seg_bf16.restype = ctypes.c_int
+    L.mua_oracle_num_blocks.argtypes = [P, i32, i32]
+    L.mua_oracle_num_blocks.restype = i64
+    return L
 
 
 def _ptr(a: np.ndarray | None):
@@ -194,7 +220,7 @@ def new_state(d: int, Bd: int, kb: int, m: int, segments=None) -> OracleState:
 
 def step(st: OracleState, p: np.ndarray, g_bits: np.ndarray, *, lr: float, beta1: float,
          beta2: float, eps: float, wd: float, t: int, seed: int,
-         want_stats: bool = False, p_exact: np.ndarray | None = None):
+         want_stats: bool = False, p_exact: np.ndarray | None = None, openmp: bool = False):
     """One MicroAdam step in place on ``st`` and ``p``.
 
     ``p`` holds the parameters: float32[d], or uint16[d] bf16 bits (each changed
@@ -202,8 +228,9 @@ def step(st: OracleState, p: np.ndarray, g_bits: np.ndarray, *, lr: float, beta1
     the values before that rounding). ``g_bits`` is the bf16 gradient as
     uint16 bits. The fp32 hyper-parameters are widened exactly to fp64.
     Returns ``(m_hat, v_hat, m_abs)`` as fp64 arrays when ``want_stats`` is
-    set, else None.
+    set, else None. ``openmp``: run the OpenMP build (same results).
     """
+    L = lib_openmp() if openmp else lib()
     assert p.dtype in (np.float32, np.uint16) and p.size == st.d and p.flags["C_CONTIGUOUS"]
     g_bits = np.ascontiguousarray(g_bits, dtype=np.uint16)
     assert g_bits.size == st.d
@@ -217,15 +244,15 @@ def step(st: OracleState, p: np.ndarray, g_bits: np.ndarray, *, lr: float, beta1
     if p.dtype == np.uint16:
         if p_exact is not None:
             assert p_exact.dtype == np.float64 and p_exact.size == st.d
-        rc = lib().mua_oracle_step_seg_bf16(_ptr(segs), segs.size, st.Bd, st.kb, st.m, _ptr(p),
+        rc = L.mua_oracle_step_seg_bf16(_ptr(segs), segs.size, st.Bd, st.kb, st.m, _ptr(p),
                                             _ptr(p_exact), _ptr(g_bits), _ptr(st.codes),
                                             _ptr(st.scal), _ptr(st.G_idx), _ptr(st.G_val), *tail)
     elif st.segs is None:
-        rc = lib().mua_oracle_step(st.d, st.Bd, st.kb, st.m, _ptr(p), _ptr(g_bits),
+        rc = L.mua_oracle_step(st.d, st.Bd, st.kb, st.m, _ptr(p), _ptr(g_bits),
                                    _ptr(st.codes), _ptr(st.scal), _ptr(st.G_idx),
                                    _ptr(st.G_val), *tail)
     else:
-        rc = lib().mua_oracle_step_seg(_ptr(st.segs), st.segs.size, st.Bd, st.kb, st.m,
+        rc = L.mua_oracle_step_seg(_ptr(st.segs), st.segs.size, st.Bd, st.kb, st.m,
                                        _ptr(p), _ptr(g_bits), _ptr(st.codes), _ptr(st.scal),
                                        _ptr(st.G_idx), _ptr(st.G_val), *tail)
     if rc != 0:

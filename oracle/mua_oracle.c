@@ -6,6 +6,13 @@
  * of the benchmark do. It shares no code, header, table or constant generator
  * with the CUDA path.
  *
+ * Built twice from this one source: plain (single-threaded) and with
+ * -fopenmp, where the `omp` annotations spread independent blocks and
+ * elements over threads. Every result is the same bit for bit in both: each
+ * block's Top-k and each element's code are computed alone, min / max are
+ * exact in any order, and every AdamStats sum adds its terms in the same
+ * age order.
+ *
  * Citations: [MicroAdam ¶n] is paragraph n of the web page "MicroAdam
  * (Sparse-Gradient Adaptive Optimization with Quantized Error Feedback)":
  *   ¶1 the per-step algorithm, ¶2 the state-memory formula, ¶3 Lemma 1 /
@@ -163,16 +170,20 @@ void mua_oracle_dequantize(const uint8_t* codes, int64_t n, float delta, float D
 void mua_oracle_quantize(const float* x, int64_t n, int64_t base, float delta, float Delta,
                          int64_t t, uint64_t seed, uint8_t* codes) {
     float inv16 = (Delta == delta) ? 0.0f : (15.0f / (Delta - delta)) * 65536.0f;
-    for (int64_t i = 0; i < n; ++i) {
-        float s16 = (x[i] - delta) * inv16;
-        uint32_t r = mua_oracle_draw16(seed, t, base + i);
-        unsigned c = 15u;
-        if (s16 >= 0.0f && s16 < 8388608.0f) {
-            uint32_t S = (uint32_t)floorf(s16);
-            uint32_t q = (S + r) >> 16;
-            c = (q > 15u) ? 15u : q;
+    /* one byte (two elements) per iteration: no two iterations share a byte */
+    #pragma omp parallel for schedule(static)
+    for (int64_t i2 = 0; i2 < (n + 1) / 2; ++i2) {
+        for (int64_t i = 2 * i2; i < 2 * i2 + 2 && i < n; ++i) {
+            float s16 = (x[i] - delta) * inv16;
+            uint32_t r = mua_oracle_draw16(seed, t, base + i);
+            unsigned c = 15u;
+            if (s16 >= 0.0f && s16 < 8388608.0f) {
+                uint32_t S = (uint32_t)floorf(s16);
+                uint32_t q = (S + r) >> 16;
+                c = (q > 15u) ? 15u : q;
+            }
+            put_code(codes, i, c);
         }
-        put_code(codes, i, c);
     }
 }
 
@@ -246,17 +257,22 @@ static int step_impl(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, 
     const float delta_t = scal[0], Delta_t = scal[1];
 
     float* a = (float*)malloc(sizeof(float) * (size_t)d);
-    keyed_t* order = (keyed_t*)malloc(sizeof(keyed_t) * (size_t)Bd);
     double* z1 = (double*)calloc((size_t)d, sizeof(double));
     double* z2 = (double*)calloc((size_t)d, sizeof(double));
     double* za = (double*)calloc((size_t)d, sizeof(double));
     uint8_t* touched = (uint8_t*)calloc((size_t)d, 1);
     int64_t* bstart = (int64_t*)malloc(sizeof(int64_t) * (size_t)nb);
     int64_t* blen = (int64_t*)malloc(sizeof(int64_t) * (size_t)nb);
-    if (!a || !order || !z1 || !z2 || !za || !touched || !bstart || !blen) {
-        free(a); free(order); free(z1); free(z2); free(za); free(touched);
-        free(bstart); free(blen);
-        return -1;
+    float* bmin = (float*)malloc(sizeof(float) * (size_t)nb);
+    float* bmax = (float*)malloc(sizeof(float) * (size_t)nb);
+    const int64_t rows = (t < m) ? t : m;
+    double* wr1 = (double*)malloc(sizeof(double) * (size_t)rows);
+    double* wr2 = (double*)malloc(sizeof(double) * (size_t)rows);
+    int failed = 0;
+    if (!a || !z1 || !z2 || !za || !touched || !bstart || !blen || !bmin || !bmax || !wr1 ||
+        !wr2) {
+        failed = 1;
+        goto done;
     }
     /* The blocks, in order: segment by segment, B_d at a time. */
     {
@@ -273,6 +289,7 @@ static int step_impl(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, 
     /* (1) a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t). */
     {
         float unit = (Delta_t - delta_t) / 15.0f;
+        #pragma omp parallel for schedule(static)
         for (int64_t i = 0; i < d; ++i) {
             float level = (float)get_code(codes, i) * unit;
             float deq = delta_t + level;
@@ -281,39 +298,59 @@ static int step_impl(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, 
     }
 
     /* (2) (I_t, V_t) = T_k(|a_t|) per block, written to row t mod m of G;
-     * (3) the selected entries of a_t are set to zero. */
+     * (3) the selected entries of a_t are set to zero; each block's residual
+     * min and max are kept for (4). */
     const int64_t row = t % m;
-    for (int64_t j = 0; j < nb; ++j) {
-        const int64_t start = bstart[j];
-        const int64_t L = blen[j];
-        const int64_t k = mua_oracle_block_k(L, Bd, kb);
-        for (int64_t q = 0; q < L; ++q) {
-            order[q].key = bits_from_f32(a[start + q]) & 0x7FFFFFFFu;
-            order[q].idx = (int32_t)q;
-        }
-        qsort(order, (size_t)L, sizeof(keyed_t), by_key_desc_idx_asc);
-        qsort(order, (size_t)k, sizeof(keyed_t), by_idx_asc);
-        int16_t* ri = G_idx + (row * nb + j) * kb;
-        uint16_t* rv = G_val + (row * nb + j) * kb;
-        for (int64_t s = 0; s < kb; ++s) {
-            if (s < k) {
-                int64_t q = order[s].idx;
-                ri[s] = (int16_t)q;
-                rv[s] = mua_oracle_f32_to_bf16(a[start + q]);
-            } else {
-                ri[s] = -1;
-                rv[s] = 0;
+    #pragma omp parallel
+    {
+        keyed_t* order = (keyed_t*)malloc(sizeof(keyed_t) * (size_t)Bd);
+        #pragma omp for schedule(dynamic, 16)
+        for (int64_t j = 0; j < nb; ++j) {
+            if (!order) {
+                failed = 1;
+                continue;
             }
+            const int64_t start = bstart[j];
+            const int64_t L = blen[j];
+            const int64_t k = mua_oracle_block_k(L, Bd, kb);
+            for (int64_t q = 0; q < L; ++q) {
+                order[q].key = bits_from_f32(a[start + q]) & 0x7FFFFFFFu;
+                order[q].idx = (int32_t)q;
+            }
+            qsort(order, (size_t)L, sizeof(keyed_t), by_key_desc_idx_asc);
+            qsort(order, (size_t)k, sizeof(keyed_t), by_idx_asc);
+            int16_t* ri = G_idx + (row * nb + j) * kb;
+            uint16_t* rv = G_val + (row * nb + j) * kb;
+            for (int64_t s = 0; s < kb; ++s) {
+                if (s < k) {
+                    int64_t q = order[s].idx;
+                    ri[s] = (int16_t)q;
+                    rv[s] = mua_oracle_f32_to_bf16(a[start + q]);
+                } else {
+                    ri[s] = -1;
+                    rv[s] = 0;
+                }
+            }
+            for (int64_t s = 0; s < k; ++s) a[start + order[s].idx] = 0.0f;
+            float lo = a[start], hi = a[start];
+            for (int64_t q = 1; q < L; ++q) {
+                if (a[start + q] < lo) lo = a[start + q];
+                if (a[start + q] > hi) hi = a[start + q];
+            }
+            bmin[j] = lo;
+            bmax[j] = hi;
         }
-        for (int64_t s = 0; s < k; ++s) a[start + order[s].idx] = 0.0f;
+        free(order);
     }
+    if (failed) goto done;
 
     /* (4) e_{t+1} = Q(a_t, delta_{t+1}, Delta_{t+1}) with the scalar min and
-     * max of the residual (a -0 result is stored as +0). */
-    float lo = a[0], hi = a[0];
-    for (int64_t i = 1; i < d; ++i) {
-        if (a[i] < lo) lo = a[i];
-        if (a[i] > hi) hi = a[i];
+     * max of the residual over all d (exact in any order; a -0 result is
+     * stored as +0). */
+    float lo = bmin[0], hi = bmax[0];
+    for (int64_t j = 1; j < nb; ++j) {
+        if (bmin[j] < lo) lo = bmin[j];
+        if (bmax[j] > hi) hi = bmax[j];
     }
     lo = lo + 0.0f;
     hi = hi + 0.0f;
@@ -323,22 +360,26 @@ static int step_impl(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, 
 
     /* (5) m_hat = AdamStats(beta1, G), v_hat = AdamStats(beta2, G^2) by the
      * unrolled decay z[I] += beta^r V over the rows in the window, oldest
-     * (largest age r) first. */
-    const int64_t rows = (t < m) ? t : m;
-    for (int64_t r = rows - 1; r >= 0; --r) {
-        const int64_t rr = (t - r) % m;
+     * (largest age r) first at every index. */
+    for (int64_t r = 0; r < rows; ++r) {
         const double w1 = pow(beta1, (double)r);
         const double w2 = pow(beta2, (double)r);
-        for (int64_t j = 0; j < nb; ++j) {
+        wr1[r] = w1;
+        wr2[r] = w2;
+    }
+    #pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < nb; ++j) {
+        for (int64_t r = rows - 1; r >= 0; --r) {
+            const int64_t rr = (t - r) % m;
             const int16_t* ri = G_idx + (rr * nb + j) * kb;
             const uint16_t* rv = G_val + (rr * nb + j) * kb;
             for (int64_t s = 0; s < kb; ++s) {
                 if (ri[s] < 0) continue;
                 const int64_t q = bstart[j] + ri[s];
                 const double V = (double)mua_oracle_bf16_to_f32(rv[s]);
-                z1[q] += w1 * V;
-                z2[q] += w2 * (V * V);
-                za[q] += w1 * fabs(V);
+                z1[q] += wr1[r] * V;
+                z2[q] += wr2[r] * (V * V);
+                za[q] += wr1[r] * fabs(V);
                 touched[q] = 1;
             }
         }
@@ -348,6 +389,7 @@ static int step_impl(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, 
 
     /* (6) p <- p*(1 - lr*wd) - lr * m_hat / (eps + sqrt(v_hat)). */
     const double decay = 1.0 - lr * wd;
+    #pragma omp parallel for schedule(static)
     for (int64_t q = 0; q < d; ++q) {
         const double m_hat = f1 * z1[q];
         const double v_hat = f2 * z2[q];
@@ -364,9 +406,10 @@ static int step_impl(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, 
         }
     }
 
-    free(a); free(order); free(z1); free(z2); free(za); free(touched);
-    free(bstart); free(blen);
-    return 0;
+done:
+    free(a); free(z1); free(z2); free(za); free(touched);
+    free(bstart); free(blen); free(bmin); free(bmax); free(wr1); free(wr2);
+    return failed ? -1 : 0;
 }
 
 int mua_oracle_step_seg(const int64_t* seg, int32_t n_seg, int32_t Bd, int32_t kb, int32_t m,

@@ -68,8 +68,8 @@ MUTANTS = {
         "const double f1 = (1.0 - beta1) / (1.0 - pow(beta1, (double)t));",
         "const double f1 = (1.0 - beta1);"),
     "vhat_of_abs_not_square": (
-        "z2[q] += w2 * (V * V);",
-        "z2[q] += w2 * fabs(V);"),
+        "z2[q] += wr2[r] * (V * V);",
+        "z2[q] += wr2[r] * fabs(V);"),
     "update_sign_flipped": (
         "pq = pq - lr * (m_hat / (eps + sqrt(v_hat)));",
         "pq = pq + lr * (m_hat / (eps + sqrt(v_hat)));"),
