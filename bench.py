@@ -5,7 +5,9 @@ Default workload: the LLaMA-2-7B-shaped parameter list (d = 6,738,415,616)
 with bf16 Student-t(3) gradients scaled per tensor, B_d = 16384, k_b = 164,
 m = 10, b = 4 (synthetic: random-init parameters, no dataset or weights).
 
-One step = mua_step = select kernel + apply kernel over the whole vector.
+One step = mua_step over the whole vector: one fused launch when every block
+of the vector fits the GPU at once (small vectors), else select kernel + apply
+kernel.
 Timing: W warm-up steps, then K steps bracketed by a barrier and a device
 synchronize, timed with CUDA events on the launching stream; with N > 1 ranks
 the vector is sharded by blocks and the ranks combine their (delta, Delta)
@@ -15,10 +17,11 @@ is the max over ranks. Inputs (47 GB) are far larger than L2 (126 MB).
 Other arms:
   --impl reference   the CPU oracle (oracle/), timed on the host cores on a
                      bounded sample of the same workload (rank 0 only).
-The JSON line also carries `roofline` (dominant kernel, algorithmic bytes per
-launch over its CUDA-event duration, against the measured HBM copy peak),
-`cpu_baseline` (the oracle on a bounded sample) and `e2e` (host-resident
-gradients copied in every step, scalars read back).
+The JSON line also carries `roofline` (the step's algorithmic bytes, 3d + 4K
++ 4mK + 8U, over its CUDA-event time, against the measured HBM copy peak, and
+per kernel its own share of those bytes, the bytes it moves and its measured
+DRAM traffic), `cpu_baseline` (the oracle on a bounded sample) and `e2e`
+(host-resident gradients copied in every step, scalars read back).
 """
 from __future__ import annotations
 
@@ -46,12 +49,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="llama2_7b",
-                    help="llama2_7b | llama2_7b_per_tensor | flat_134m | flat_1m | bert_base | "
-                         "bert_base_<B_d>[_per_tensor] | flat_1g_m<m>")
+                    help="llama2_7b | llama2_7b_bf16 | llama2_7b_per_tensor | flat_134m | flat_1m | "
+                         "bert_base | bert_base_<B_d>[_per_tensor] | flat_1g_m<m>")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--update-split", type=int, default=None,
-                    help="eighths of the blocks whose parameter update runs in the select kernel")
     ap.add_argument("--wd", type=float, default=None,
                     help="weight decay instead of the workload's (AdamW-style, every parameter)")
     ap.add_argument("--cpu-sample", type=int, default=1 << 23,
@@ -69,6 +70,9 @@ def _named_workload(name):
     from compressed_state_optimizer_b200 import workloads as W
     if name == "llama2_7b":
         return W.llama2_7b()
+    if name == "llama2_7b_bf16":
+        import dataclasses
+        return dataclasses.replace(W.llama2_7b(), name="llama2_7b_bf16", params="bf16")
     if name == "llama2_7b_per_tensor":
         import dataclasses
         return dataclasses.replace(W.llama2_7b(), name="llama2_7b_per_tensor", per_tensor=True)
@@ -211,29 +215,54 @@ def union_size(window_u32, nb, m, kp, Bd, d, torch):
     return total
 
 
-def cpu_baseline(w, sample: int, max_seconds: float = 12.0, min_steps: int = 2):
-    """The oracle as it stands on the first `sample` parameters of the workload."""
-    import numpy as np
+def host_info():
+    """Host cores and RAM of this box (for the CPU legs' records)."""
+    cores = os.cpu_count() or 1
+    try:
+        ram = int(re.search(r"MemTotal:\s+(\d+)", open("/proc/meminfo").read()).group(1)) * 1024
+    except Exception:
+        ram = None
+    return cores, ram
+
+
+def _time_oracle(w, n: int, openmp: bool, max_seconds: float, min_steps: int = 2):
+    """Steps t = 1, 2, ... of the oracle on the first n parameters of the
+    workload until max_seconds of oracle time (gradient generation excluded)."""
     import oracle
     from compressed_state_optimizer_b200 import workloads as W
-    n = min(sample, w.d)
     p = W.make_params(n, seed=7).numpy().copy()
     st = oracle.new_state(n, w.Bd, w.kb, w.m)
-    steps, t0 = 0, time.perf_counter()
-    elapsed = 0.0
+    steps, elapsed, t0 = 0, 0.0, time.perf_counter()
     while steps < min_steps or elapsed < max_seconds:
         g = W.bf16_bits(W.make_grads(w, steps + 1, start=0, length=n))
         s0 = time.perf_counter()
         oracle.step(st, p, g, lr=w.lr, beta1=w.beta1, beta2=w.beta2, eps=w.eps, wd=w.wd,
-                    t=steps + 1, seed=w.seed)
+                    t=steps + 1, seed=w.seed, openmp=openmp)
         elapsed += time.perf_counter() - s0
         steps += 1
         if time.perf_counter() - t0 > 4 * max_seconds:
             break
-    return {"value": n * steps / elapsed / 1e9, "unit": "Gparams/s", "cores": 1,
-            "kind": "oracle",
-            "sample": f"first {n} parameters of {w.name}, {steps} steps "
-                      f"(t=1..{steps}), single-threaded C oracle, {elapsed:.1f} s"}
+    return n * steps / elapsed / 1e9, steps, elapsed
+
+
+def cpu_baseline(w, sample: int, max_seconds: float = 12.0):
+    """The oracle as it stands on the first `sample` parameters of the workload:
+    its OpenMP build on every host core (the headline) and the plain
+    single-threaded build (a sub-record)."""
+    import oracle
+    n = min(sample, w.d)
+    cores, ram = host_info()
+    oracle.set_threads(cores)
+    v_omp, s_omp, e_omp = _time_oracle(w, n, True, max_seconds)
+    v_one, s_one, e_one = _time_oracle(w, n, False, max_seconds / 2)
+    return {"value": v_omp, "unit": "Gparams/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} parameters of {w.name}, {s_omp} steps (t=1..{s_omp}), "
+                      f"C oracle built with OpenMP over blocks, {cores} threads, "
+                      f"{e_omp:.1f} s",
+            "host_ram_bytes": ram,
+            "single_thread": {"value": v_one, "unit": "Gparams/s", "cores": 1,
+                              "sample": f"first {n} parameters, {s_one} steps, plain build, "
+                                        f"{e_one:.1f} s"}}
 
 
 # --------------------------------------------------------------------- reference arm
@@ -244,10 +273,13 @@ def run_reference(args, rank, world):
     n = min(args.cpu_sample, w.d)
     import oracle
     from compressed_state_optimizer_b200 import workloads as W
+    cores, ram = host_info()
+    oracle.set_threads(cores)
     p = W.make_params(n, seed=7).numpy().copy()
     st = oracle.new_state(n, w.Bd, w.kb, w.m)
     grads = [W.bf16_bits(W.make_grads(w, s, start=0, length=n)) for s in (1, 2)]
-    hyper = dict(lr=w.lr, beta1=w.beta1, beta2=w.beta2, eps=w.eps, wd=w.wd, seed=w.seed)
+    hyper = dict(lr=w.lr, beta1=w.beta1, beta2=w.beta2, eps=w.eps, wd=w.wd, seed=w.seed,
+                 openmp=True)
     t = 0
     for _ in range(args.warmup):
         t += 1
@@ -264,8 +296,10 @@ def run_reference(args, rank, world):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "d": w.d, "B_d": w.Bd, "k_b": w.kb, "m": w.m, "b": 4, "wd": w.wd,
                        "sample_params": n, "l2": "host run"},
-            "cpu_baseline": {"value": value, "unit": "Gparams/s", "cores": 1, "kind": "oracle",
-                             "sample": f"first {n} parameters of {w.name} per step"},
+            "cpu_baseline": {"value": value, "unit": "Gparams/s", "cores": cores, "kind": "oracle",
+                             "sample": f"first {n} parameters of {w.name} per step, C oracle "
+                                       f"built with OpenMP over blocks, {cores} threads",
+                             "host_ram_bytes": ram},
             "e2e": {"value": value, "unit": "Gparams/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -285,10 +319,10 @@ def run_ours(args, rank, world, local_rank):
         raise SystemExit("the per-tensor cut runs on one GPU")
     mo = MicroAdam(w.d, block_size=w.Bd, k_per_block=w.kb, window=w.m, segments=segs,
                    shard=None if world == 1 else sharding.shard_blocks(w.d, w.Bd, rank, world))
-    if args.update_split is not None:
-        mo.set_update_split(args.update_split)
     d_loc, off = mo.d, mo.offset
     params = W.make_params(d_loc, seed=7 + rank, device=dev)
+    if w.params == "bf16":
+        params = params.to(torch.bfloat16)
     grads = [W.make_grads(w, s, device=dev, start=off, length=d_loc) for s in (1, 2)]
     state = mo.new_state(dev)
     stream = torch.cuda.current_stream(dev)
@@ -313,30 +347,60 @@ def run_ours(args, rank, world, local_rank):
         step(t, grads[t % 2])
     barrier()
 
-    # ---- timed region: K full steps, with per-kernel events on the same stream.
+    # ---- timed region: K full steps (mua_step at N = 1; select, the 8-byte
+    # all-reduce and apply at N > 1), each bracketed by events on the launching
+    # stream. A working set that fits in L2 is flushed from it before every step (a
+    # write of twice L2's size, outside the events around the step); larger
+    # ones are streamed from HBM anyway.
+    work_bytes = params.element_size() * d_loc + 2 * 2 * d_loc + mo.state_bytes
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = None
+    if work_bytes < 4 * l2_bytes:
+        flush = torch.empty(2 * l2_bytes // 4, dtype=torch.int32, device=dev)
     clocks = ClockSampler(gpu_id(dev))
     clocks.start()
     time.sleep(0.3)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     start.record(stream)
     for i in range(args.steps):
         t += 1
-        g = grads[t % 2]
+        if flush is not None:
+            flush.fill_(i)
         ev[i][0].record(stream)
-        mo.select(params, g, state, t=t, **hyper)
+        step(t, grads[t % 2])
         ev[i][1].record(stream)
-        if world > 1:
-            sharding.combine_minmax_(state, mo.minmax_offset(t))
-        mo.apply(params, g, state, t=t, **hyper)
-        ev[i][2].record(stream)
     end.record(stream)
     barrier()
     clk = clocks.stop()
-    total_ms = start.elapsed_time(end)
-    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    app_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    if flush is None:
+        total_ms = start.elapsed_time(end)
+    else:  # the steps alone, without the flushes between them
+        total_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+
+    # ---- per-kernel breakdown (outside the timed region): the two-kernel
+    # path's select and apply, each timed on the launching stream.
+    launches = 2 if world > 1 else mo.step_launches(bf16_params=w.params == "bf16")
+    nb_steps = max(3, min(10, args.steps))
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nb_steps)]
+    barrier()
+    for i in range(nb_steps):
+        t += 1
+        g = grads[t % 2]
+        if flush is not None:
+            flush.fill_(i)
+        kev[i][0].record(stream)
+        mo.select(params, g, state, t=t, **hyper)
+        kev[i][1].record(stream)
+        if world > 1:
+            sharding.combine_minmax_(state, mo.minmax_offset(t))
+        mo.apply(params, g, state, t=t, **hyper)
+        kev[i][2].record(stream)
+    barrier()
+    sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in kev)
+    app_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in kev)
+    fused_ms = total_ms / args.steps if launches == 1 else None
     if world > 1:
         tm = torch.tensor([total_ms], device=dev)
         dist.all_reduce(tm, op=dist.ReduceOp.MAX)
@@ -344,7 +408,11 @@ def run_ours(args, rank, world, local_rank):
     ms_per_step = total_ms / args.steps
     value = w.d / (ms_per_step * 1e-3) / 1e9
 
-    # ---- algorithmic bytes (per launch, this rank's shard)
+    # ---- algorithmic bytes per step (this rank's shard): the method's bytes,
+    # each kernel billed for its own share of them (select: g, e read, new row
+    # written; apply: e written, window read, parameter read-modify-write on
+    # the window's index union), and what each kernel must move in this
+    # two-kernel design (apply re-reads g and e to recompute a_t).
     lay = mo.layout
     nb = lay.blocks
     if segs is None:
@@ -355,15 +423,34 @@ def run_ours(args, rank, world, local_rank):
     win = state[lay.window: lay.window + 4 * nb * w.m * lay.row_stride].view(torch.int32)
     U = union_size(win, nb, w.m, lay.row_stride, w.Bd, d_loc, torch)
     rows = min(t, w.m)
-    bytes_select = 2.5 * d_loc + 4 * K
-    bytes_apply = 3.0 * d_loc + 4 * rows * K + 8 * U
-    bytes_step = 2.0 * d_loc + 1.0 * d_loc + 4 * K + 4 * rows * K + 8 * U
+    # parameter read-modify-write: the union (and, with weight decay, every parameter)
+    rmw = 2 * params.element_size() * (d_loc if w.wd else U)
+    own = {"select": 2.5 * d_loc + 4 * K, "apply": 0.5 * d_loc + 4 * rows * K + rmw}
+    moved = {"select": 2.5 * d_loc + 4 * K, "apply": 3.0 * d_loc + 4 * rows * K + rmw}
+    bytes_step = own["select"] + own["apply"]  # 3 d + 4 K + 4 rows K + 8 U (fp32, wd = 0)
     peak, peak_kind = measured_peak()
-    dominant = "apply" if app_ms >= sel_ms else "select"
-    dom_ms = max(app_ms, sel_ms)
-    dom_bytes = bytes_apply if dominant == "apply" else bytes_select
-    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
-    traffic = profiled_traffic(dominant, w.name)
+    kms = {"select": sel_ms, "apply": app_ms}
+    kernels = {}
+    traffic_step = 0.0
+    for kname in ("select", "apply"):
+        tr = profiled_traffic(kname, w.name)
+        kernels[kname] = {
+            "ms": kms[kname], "bytes": own[kname],
+            "frac": own[kname] / (kms[kname] * 1e-3) / 1e9 / peak,
+            "bytes_moved": moved[kname],
+            "frac_moved": moved[kname] / (kms[kname] * 1e-3) / 1e9 / peak,
+            "traffic": tr,
+            "dram_frac": None if tr is None else tr / (kms[kname] * 1e-3) / 1e9 / peak}
+        traffic_step = None if (tr is None or traffic_step is None) else traffic_step + tr
+    if fused_ms is not None:  # one launch moves the method's bytes only (no re-read)
+        tr = profiled_traffic("fused", w.name)
+        kernels["fused"] = {"ms": fused_ms, "bytes": bytes_step,
+                            "frac": bytes_step / (fused_ms * 1e-3) / 1e9 / peak,
+                            "bytes_moved": bytes_step, "traffic": tr,
+                            "dram_frac": None if tr is None else tr / (fused_ms * 1e-3) / 1e9 / peak}
+        traffic_step = tr
+    achieved = bytes_step * world / (ms_per_step * 1e-3) / 1e9
+    dominant = "fused" if fused_ms is not None else ("apply" if app_ms >= sel_ms else "select")
 
     # ---- end to end: gradients from pinned host memory every step, scalars back.
     e2e = None
@@ -377,17 +464,25 @@ def run_ours(args, rank, world, local_rank):
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": w.name, "d": w.d, "B_d": w.Bd, "k_b": w.kb, "m": w.m, "wd": w.wd,
+                       "params": w.params,
                        "blocks": "per tensor" if segs is not None else "over the flat vector",
                        "b": 4, "grads": w.grad, "parallelism": f"blocks sharded over {world}"
                        if world > 1 else "single GPU",
-                       "l2": "inputs (params+grads+state ~47 GB) larger than L2"},
-            "hbm_gbs_algorithmic_step": bytes_step * world / (ms_per_step * 1e-3) / 1e9,
-            "kernels_ms": {"select": sel_ms, "apply": app_ms},
+                       "l2": (f"working set {work_bytes / 1e9:.2f} GB > L2; no flush"
+                              if flush is None else
+                              f"working set {work_bytes / 1e6:.1f} MB fits L2: flushed "
+                              f"({2 * l2_bytes >> 20} MiB write) before every step, outside "
+                              "the timed events")},
+            "kernels_ms": dict({"select": sel_ms, "apply": app_ms},
+                               **({"fused": fused_ms} if fused_ms is not None else {})),
+            "step_path": "one fused launch" if launches == 1 else "select + apply",
             "union_fraction": U / d_loc,
-            "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": traffic, "algorithmic_bytes": dom_bytes},
-            "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "hbm", "kernel": "step (select + apply)", "achieved": achieved,
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak, "step_frac": achieved / peak,
+                         "traffic": traffic_step, "algorithmic_bytes": bytes_step,
+                         "dominant_kernel": dominant, "kernels": kernels},
+            "gpu_launches": launches * args.steps,
             "clocks": clk,
         }
         if e2e is not None:

@@ -38,12 +38,16 @@ SIGNATURES = {
     "mua_step": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P]),
     "mua_select": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P,
                                   _P, _P]),
-    "mua_set_update_split": (ctypes.c_int, [_P, _i32]),
-    "mua_set_select_variant": (ctypes.c_int, [_P, _i32]),
     "mua_minmax_offset": (_i64, [_P, _i64]),
     "mua_apply": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64, _P,
                                  _P, _P]),
-    "mua_get_status": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_uint32), _P]),
+    "mua_get_status": (ctypes.c_int, [_P, _P, _P, ctypes.POINTER(ctypes.c_int32)]),
+    "mua_step_launches": (ctypes.c_int, [_P, _i32]),
+    "mua_step_bf16": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64,
+                                     _P]),
+    "mua_apply_bf16": (ctypes.c_int, [_P, _P, _P, _P, _f32, _f32, _f32, _f32, _f32, _i64, _u64,
+                                      _P, _P, _P]),
+    "mua_set_wait_limit_ns": (ctypes.c_int, [_P, _i64]),
     "mua_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "mua_last_cuda_error": (ctypes.c_char_p, []),
     "mua_version": (ctypes.c_char_p, []),
@@ -171,7 +175,8 @@ class MicroAdam:
     def _check_tensors(self, params, grads, state):
         import torch
         if params is not None:
-            assert params.dtype == torch.float32 and params.is_cuda and params.is_contiguous()
+            assert params.dtype in (torch.float32, torch.bfloat16)
+            assert params.is_cuda and params.is_contiguous()
             assert params.numel() == self.d, (params.numel(), self.d)
         assert grads.dtype == torch.bfloat16 and grads.is_cuda and grads.is_contiguous()
         assert grads.numel() == self.d
@@ -179,34 +184,36 @@ class MicroAdam:
 
     # ------------------------------------------------------------ steps
     def step(self, params, grads, state, *, lr, beta1, beta2, eps, wd, t, seed, stream=None):
-        """One full step t on ``stream`` (default: the current stream)."""
+        """One full step t on ``stream`` (default: the current stream);
+        ``params`` fp32 (mua_step) or bf16 (mua_step_bf16)."""
+        import torch
         self._check_tensors(params, grads, state)
-        _check(library().mua_step(self._h, params.data_ptr(), grads.data_ptr(), state.data_ptr(),
-                                  lr, beta1, beta2, eps, wd, t, seed, _stream_ptr(stream)),
-               "mua_step")
+        name = "mua_step_bf16" if params.dtype == torch.bfloat16 else "mua_step"
+        _check(getattr(library(), name)(self._h, params.data_ptr(), grads.data_ptr(),
+                                        state.data_ptr(), lr, beta1, beta2, eps, wd, t, seed,
+                                        _stream_ptr(stream)), name)
 
     def select(self, params, grads, state, *, lr, beta1, beta2, eps, wd, t, seed, mhat=None,
                vhat=None, stream=None):
-        """First half of step t (Top-k, window row, min/max partials, and the
-        parameter update of the blocks the select kernel owns)."""
+        """First half of step t (Top-k, window row, min/max partials)."""
         self._half("mua_select", params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
                    vhat, stream)
 
-    def set_select_variant(self, variant: int):
-        """0: one warp per block (default); 1: one CTA per block; 2: persistent CTAs."""
-        _check(library().mua_set_select_variant(self._h, int(variant)), "mua_set_select_variant")
-
-    def set_update_split(self, split: int):
-        _check(library().mua_set_update_split(self._h, split), "mua_set_update_split")
-
     def _half(self, name, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat, vhat,
               stream):
+        import torch
         self._check_tensors(params, grads, state)
+        if params is not None and params.dtype == torch.bfloat16:
+            if name == "mua_select":
+                params = None  # not touched by the select kernel
+            else:
+                name = name + "_bf16"
         for x in (mhat, vhat):
             if x is not None:
                 assert x.is_cuda and x.numel() == self.d and x.is_contiguous()
         fn = getattr(library(), name)
-        _check(fn(self._h, params.data_ptr(), grads.data_ptr(), state.data_ptr(), lr, beta1,
+        _check(fn(self._h, params.data_ptr() if params is not None else None, grads.data_ptr(),
+                  state.data_ptr(), lr, beta1,
                   beta2, eps, wd, t, seed, mhat.data_ptr() if mhat is not None else None,
                   vhat.data_ptr() if vhat is not None else None, _stream_ptr(stream)), name)
 
@@ -218,13 +225,24 @@ class MicroAdam:
 
     def apply(self, params, grads, state, *, lr, beta1, beta2, eps, wd, t, seed, mhat=None,
               vhat=None, stream=None):
-        """Second half of step t (4-bit quantization of the residual, and the
-        parameter update of the remaining blocks)."""
+        """Second half of step t (4-bit quantization of the residual and the
+        AdamStats update of the parameters)."""
         self._half("mua_apply", params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
                    vhat, stream)
 
+    def step_launches(self, bf16_params: bool = False) -> int:
+        """Kernel launches of one ``step`` on the current device (1: fused)."""
+        n = int(library().mua_step_launches(self._h, 1 if bf16_params else 0))
+        if n < 0:
+            raise MuaError(n, "mua_step_launches")
+        return n
+
+    def set_wait_limit_ns(self, ns: int):
+        """Bound on the fused step's grid-barrier wait (<= 0: give up at once)."""
+        _check(library().mua_set_wait_limit_ns(self._h, int(ns)), "mua_set_wait_limit_ns")
+
     def status(self, state, stream=None) -> int:
-        out = ctypes.c_uint32()
-        _check(library().mua_get_status(self._h, state.data_ptr(), ctypes.byref(out),
-                                        _stream_ptr(stream)), "mua_get_status")
+        out = ctypes.c_int32()
+        _check(library().mua_get_status(self._h, state.data_ptr(), _stream_ptr(stream),
+                                        ctypes.byref(out)), "mua_get_status")
         return int(out.value)

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmua.so")
-SOURCES = ["mua_api.cu", "mua_select.cu", "mua_select_warp.cu", "mua_apply.cu"]
+SOURCES = ["mua_api.cu", "mua_select_warp.cu", "mua_apply.cu", "mua_fused.cu"]
 HEADERS = ["mua_kernels.cuh", os.path.join("..", "..", "include", "mua.h")]
 
 NVCC_FLAGS = [

@@ -5,12 +5,10 @@
 //
 // A handle holds geometry only. mua_step enqueues, on the caller's stream:
 //   1. an 8-byte memset of the (-delta_{t+1}, Delta_{t+1}) accumulator pair,
-//   2. the select kernel: by default one warp per block (mua_select_warp.cu);
-//      the CTA shapes of mua_select.cu (variants 1, 2) can also update the
-//      parameters of the blocks with (j & 7) < update_split,
-//   3. the apply kernel (one CTA of half the select CTA's threads per block,
-//      reverse block order so the tail of the select kernel's reads is still
-//      in L2): codec, then the AdamStats update of the remaining blocks.
+//   2. the select kernel, one warp per block (mua_select_warp.cu),
+//   3. the apply kernel (one CTA per block, reverse block order so the tail
+//      of the select kernel's reads is still in L2): codec, then the
+//      AdamStats update of the block (mua_apply.cu).
 // Everything the kernels need per step (beta^r weights, bias corrections,
 // Philox round keys) is computed here in fp64 and rounded once to fp32 /
 // uint32 before launch.
@@ -32,14 +30,13 @@ struct mua_ctx {
   int64_t nb;           // blocks of this handle
   int32_t Bd, kb, kp, m;
   int32_t last_len;
-  int32_t threads;       // CTA size of the select variants (32 elements per thread)
   int32_t apply_threads; // CTA size of the apply kernel (two passes per block from B_d 2048)
   bool vec;             // 16-byte vector path usable (B_d % 8 == 0)
-  bool persistent;      // bulk-copy pipelined kernels usable (B_d % 32 == 0)
-  int32_t variant;      // select kernel: 0 warp per block, 1 CTA per block, 2 persistent CTAs
   int64_t off_codes, off_window, bytes;
-  uint32_t select_smem, apply_smem;
-  int32_t update_split;  // blocks with (j & 7) < split update in the select kernel
+  uint32_t apply_smem;
+  bool whole;           // the handle covers the whole vector (not one shard of it)
+  int64_t wait_ns;      // bound on a grid-barrier wait (fused step)
+  int32_t fused_cap[2][mua::kMaxDevices];  // co-resident fused CTAs [bf16][device] (-1: unknown)
   // Tensor list cut per tensor (n_seg > 0; whole vector, not a shard).
   int32_t n_seg;
   int32_t seg_first[mua::kMaxSegments];
@@ -49,12 +46,11 @@ struct mua_ctx {
 
 namespace {
 
-// Share of the blocks (in eighths) whose parameter update runs in the select
-// kernel: select does the arithmetic-heavy Top-k, apply the Philox codec; the
-// update is HBM traffic, placed to balance the two.
-constexpr int32_t kDefaultUpdateSplit = 4;
-
 thread_local char g_cuda_err[256] = "no CUDA error";
+
+// Default bound on the fused step's grid-barrier wait: far above a step's
+// duration, far below anything that would look like a hang.
+constexpr int64_t kDefaultWaitNs = 2000000000;
 
 int cuda_fail(cudaError_t e, const char* where) {
   std::snprintf(g_cuda_err, sizeof g_cuda_err, "%s: %s", where, cudaGetErrorString(e));
@@ -82,9 +78,10 @@ int apply_warps_per_sm(int T, int Bd, int kp, int m) {
   return std::min(by_bound, std::min(by_smem, by_threads)) * (T / 32);
 }
 
-// Half the select CTA (the block in two passes; more CTAs per SM, so one
-// CTA's update barriers overlap the others' codec) unless the update's
-// shared memory makes the full CTA keep more warps resident (long windows).
+// Half of T, the CTA that holds a block in one pass (the block then takes two
+// passes; more CTAs per SM, so one CTA's update barriers overlap the others'
+// codec work), unless the update's shared memory makes the full CTA keep more
+// warps resident (long windows).
 int pick_apply_threads(int T, int Bd, int kp, int m) {
   if (T < 64) return T;
   return apply_warps_per_sm(T / 2, Bd, kp, m) >= apply_warps_per_sm(T, Bd, kp, m) ? T / 2 : T;
@@ -118,17 +115,15 @@ int make(int64_t d_total, int32_t Bd, int32_t kb, int32_t m, int32_t bits,
   h->kp = kp;
   h->m = m;
   h->last_len = (int32_t)(h->d - (block_count - 1) * Bd);
-  h->threads = pick_threads(Bd);
-  h->apply_threads = pick_apply_threads(h->threads, Bd, kp, m);
+  h->apply_threads = pick_apply_threads(pick_threads(Bd), Bd, kp, m);
   h->vec = (Bd % 8) == 0;
-  h->persistent = false;
-  h->variant = 0;
   h->off_codes = 256;
   h->off_window = h->off_codes + round_up((h->d + 1) / 2, 256);
   h->bytes = h->off_window + 4 * block_count * (int64_t)m * kp;
-  h->select_smem = mua::select_smem_bytes(h->threads, Bd, kp, m);
   h->apply_smem = mua::apply_smem_bytes(h->apply_threads, Bd, kp, m);
-  h->update_split = kDefaultUpdateSplit;
+  h->whole = (block_begin == 0 && block_count == nb_total);
+  h->wait_ns = kDefaultWaitNs;
+  for (int i = 0; i < mua::kMaxDevices; ++i) h->fused_cap[0][i] = h->fused_cap[1][i] = -1;
   h->n_seg = 0;
   *out = h;
   return MUA_OK;
@@ -177,7 +172,9 @@ bool finite_f(float x) { return std::isfinite(x); }
 
 int check_hyper(float lr, float beta1, float beta2, float eps, float wd, int64_t t) {
   if (t < 1) return MUA_ERR_ARG;
-  if (!finite_f(lr) || !finite_f(wd) || !finite_f(eps) || eps < 0.0f) return MUA_ERR_ARG;
+  // eps > 0: with eps = 0 an index whose window values are all zero would give
+  // m_hat / sqrt(v_hat) = 0 / 0.
+  if (!finite_f(lr) || !finite_f(wd) || !finite_f(eps) || !(eps > 0.0f)) return MUA_ERR_ARG;
   if (!(beta1 >= 0.0f && beta1 < 1.0f) || !(beta2 >= 0.0f && beta2 < 1.0f)) return MUA_ERR_ARG;
   return MUA_OK;
 }
@@ -242,18 +239,23 @@ int64_t mua_minmax_offset(mua_t h, int64_t t) {
   return 4 * (int64_t)pair_word(t + 1);
 }
 
-static int fill_args(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
-                     float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
-                     float* mhat, float* vhat, mua::StepArgs* out) {
-  if (!h || !params || !grads || !state) return MUA_ERR_ARG;
+// params: fp32[d] or, with bf16, bf16[d] bits; it may be NULL only for
+// mua_select (which does not touch it).
+static int fill_args(mua_t h, void* params, bool bf16, const uint16_t* grads, void* state,
+                     float lr, float beta1, float beta2, float eps, float wd, int64_t t,
+                     uint64_t seed, float* mhat, float* vhat, mua::StepArgs* out,
+                     bool params_optional = false) {
+  if (!h || (!params && !params_optional) || !grads || !state) return MUA_ERR_ARG;
   const int rc = check_hyper(lr, beta1, beta2, eps, wd, t);
   if (rc != MUA_OK) return rc;
   if (!aligned16(params) || !aligned16(grads) || !aligned16(state)) return MUA_ERR_ALIGN;
+  if ((mhat && !aligned16(mhat)) || (vhat && !aligned16(vhat))) return MUA_ERR_ALIGN;
   uint8_t* st = static_cast<uint8_t*>(state);
   mua::StepArgs& A = *out;
   std::memset(&A, 0, sizeof A);
   A.g = geometry(h);
-  A.params = params;
+  A.params = bf16 ? nullptr : static_cast<float*>(params);
+  A.params16 = bf16 ? static_cast<uint16_t*>(params) : nullptr;
   A.grads = grads;
   A.codes = st + h->off_codes;
   A.window = reinterpret_cast<uint32_t*>(st + h->off_window);
@@ -271,10 +273,9 @@ static int fill_args(mua_t h, float* params, const uint16_t* grads, void* state,
   A.eps = eps;
   A.decay = (float)(1.0 - (double)lr * (double)wd);
   A.has_decay = (wd != 0.0f);
-  // The warp-per-block select does no parameter update: apply does them all.
-  A.update_split = (h->variant == 0) ? 0 : h->update_split;
   // Exact for e < 2^16: (2^32 mod kp) < kp and e * kp < 2^31 keep the error below 1/kp.
   A.kp_recip = (uint32_t)(((1ull << 32) + (uint64_t)h->kp - 1) / (uint64_t)h->kp);
+  A.wait_ns = (uint64_t)std::max<int64_t>(0, h->wait_ns);
   A.n_seg = h->n_seg;
   for (int32_t s = 0; s < h->n_seg; ++s) {
     A.seg_first[s] = h->seg_first[s];
@@ -285,7 +286,7 @@ static int fill_args(mua_t h, float* params, const uint16_t* grads, void* state,
   // m_hat = (1-beta1)/(1-beta1^t) * sum_r beta1^r V_r, likewise v_hat.
   A.f1 = (float)((1.0 - b1) / (1.0 - std::pow(b1, (double)t)));
   A.f2 = (float)((1.0 - b2) / (1.0 - std::pow(b2, (double)t)));
-  for (int r = 0; r < mua::kMaxWindow; ++r) {
+  for (int r = 0; r < h->m; ++r) {
     A.w1[r] = (float)std::pow(b1, (double)r);
     A.w2[r] = (float)std::pow(b2, (double)r);
   }
@@ -303,61 +304,112 @@ int mua_select(mua_t h, float* params, const uint16_t* grads, void* state, float
                float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
                float* mhat, float* vhat, void* stream) {
   mua::StepArgs A;
-  const int rc = fill_args(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
-                           vhat, &A);
+  const int rc = fill_args(h, params, false, grads, state, lr, beta1, beta2, eps, wd, t, seed,
+                           mhat, vhat, &A, /*params_optional=*/true);
   if (rc != MUA_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(A.hdr + A.pair_next, 0, 8, s);
   if (e != cudaSuccess) return cuda_fail(e, "reset of the min/max pair");
-  if (h->variant == 0)
-    e = mua::launch_select_warp(A, h->vec, s);
-  else
-    e = mua::launch_select(A, h->threads, h->vec, h->variant == 2, h->select_smem, s);
+  e = mua::launch_select_warp(A, h->vec, s);
   if (e != cudaSuccess) return cuda_fail(e, "select kernel launch");
+  return MUA_OK;
+}
+
+static int apply_impl(mua_t h, void* params, bool bf16, const uint16_t* grads, void* state,
+                      float lr, float beta1, float beta2, float eps, float wd, int64_t t,
+                      uint64_t seed, float* mhat, float* vhat, void* stream) {
+  mua::StepArgs A;
+  const int rc = fill_args(h, params, bf16, grads, state, lr, beta1, beta2, eps, wd, t, seed,
+                           mhat, vhat, &A);
+  if (rc != MUA_OK) return rc;
+  const cudaError_t e = mua::launch_apply(A, h->apply_threads, h->vec, h->apply_smem,
+                                          static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "apply kernel launch");
   return MUA_OK;
 }
 
 int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
               float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
               float* mhat, float* vhat, void* stream) {
+  return apply_impl(h, params, false, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
+                    vhat, stream);
+}
+
+int mua_apply_bf16(mua_t h, uint16_t* params, const uint16_t* grads, void* state, float lr,
+                   float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+                   float* mhat, float* vhat, void* stream) {
+  return apply_impl(h, params, true, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
+                    vhat, stream);
+}
+
+// Whether mua_step runs as one fused launch on the current device: a whole
+// vector of blocks of at most 16384 entries, all of whose CTAs the device
+// holds at once. Returns a negative MUA_ERR_CUDA code if the query fails.
+static int use_fused(mua_t h, bool bf16) {
+  if (!h->whole || h->Bd > 16384) return 0;
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "device query");
+  const bool known = dev >= 0 && dev < mua::kMaxDevices;
+  int cap = known ? h->fused_cap[bf16][dev] : -1;
+  if (cap < 0) {
+    cap = mua::fused_max_blocks(h->Bd, h->kp, h->m, h->vec, bf16);
+    if (known) h->fused_cap[bf16][dev] = cap;
+  }
+  return h->nb <= cap ? 1 : 0;
+}
+
+static int step_impl(mua_t h, void* params, bool bf16, const uint16_t* grads, void* state,
+                     float lr, float beta1, float beta2, float eps, float wd, int64_t t,
+                     uint64_t seed, void* stream) {
   mua::StepArgs A;
-  const int rc = fill_args(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, mhat,
-                           vhat, &A);
+  int rc = fill_args(h, params, bf16, grads, state, lr, beta1, beta2, eps, wd, t, seed, nullptr,
+                     nullptr, &A);
   if (rc != MUA_OK) return rc;
-  const cudaError_t e =
-      mua::launch_apply(A, h->apply_threads, h->vec, h->apply_smem, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "apply kernel launch");
+  const int fused = use_fused(h, bf16);
+  if (fused < 0) return fused;
+  if (!fused) {
+    rc = mua_select(h, nullptr, grads, state, lr, beta1, beta2, eps, wd, t, seed, nullptr,
+                    nullptr, stream);
+    if (rc != MUA_OK) return rc;
+    return apply_impl(h, params, bf16, grads, state, lr, beta1, beta2, eps, wd, t, seed,
+                      nullptr, nullptr, stream);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(A.hdr + A.pair_next, 0, 8, s);
+  if (e != cudaSuccess) return cuda_fail(e, "reset of the min/max pair");
+  e = cudaMemsetAsync(A.hdr + mua::kHdrBarrier, 0, 4, s);
+  if (e != cudaSuccess) return cuda_fail(e, "reset of the barrier word");
+  e = mua::launch_fused(A, h->vec, s);
+  if (e != cudaSuccess) return cuda_fail(e, "fused kernel launch");
   return MUA_OK;
 }
 
 int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float lr, float beta1,
              float beta2, float eps, float wd, int64_t t, uint64_t seed, void* stream) {
-  int rc = mua_select(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, nullptr,
-                      nullptr, stream);
-  if (rc != MUA_OK) return rc;
-  return mua_apply(h, params, grads, state, lr, beta1, beta2, eps, wd, t, seed, nullptr, nullptr,
-                   stream);
+  return step_impl(h, params, false, grads, state, lr, beta1, beta2, eps, wd, t, seed, stream);
 }
 
-int mua_set_select_variant(mua_t h, int32_t variant) {
-  if (!h || variant < 0 || variant > 2) return MUA_ERR_ARG;
-  if (variant == 2 && !((h->Bd % 32) == 0 && h->nb >= 2 && h->n_seg == 0))
-    return MUA_ERR_UNSUPPORTED;
-  // The CTA shapes hold the update's shared memory too (and variant 2 a copy
-  // of the block): it must fit one CTA's 227 KB beside the static arrays.
-  const uint32_t stage = variant == 2 ? ((2u * (uint32_t)h->Bd + (uint32_t)h->Bd / 2u + 127u) & ~127u) : 0u;
-  if (variant != 0 && h->select_smem + stage > 227u * 1024u - 8u * 1024u) return MUA_ERR_UNSUPPORTED;
-  h->variant = variant;
+int mua_step_bf16(mua_t h, uint16_t* params, const uint16_t* grads, void* state, float lr,
+                  float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+                  void* stream) {
+  return step_impl(h, params, true, grads, state, lr, beta1, beta2, eps, wd, t, seed, stream);
+}
+
+int mua_step_launches(mua_t h, int32_t bf16_params) {
+  if (!h) return MUA_ERR_ARG;
+  const int fused = use_fused(h, bf16_params != 0);
+  if (fused < 0) return fused;
+  return fused ? 1 : 2;
+}
+
+int mua_set_wait_limit_ns(mua_t h, int64_t ns) {
+  if (!h) return MUA_ERR_ARG;
+  h->wait_ns = ns <= 0 ? 0 : ns;
   return MUA_OK;
 }
 
-int mua_set_update_split(mua_t h, int32_t split) {
-  if (!h || split < 0 || split > 8) return MUA_ERR_ARG;
-  h->update_split = split;
-  return MUA_OK;
-}
-
-int mua_get_status(mua_t h, const void* state, uint32_t* out, void* stream) {
+int mua_get_status(mua_t h, const void* state, void* stream, int32_t* out) {
   if (!h || !state || !out) return MUA_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const uint32_t* hdr = static_cast<const uint32_t*>(state);
@@ -372,7 +424,7 @@ const char* mua_strerror(int code) {
   switch (code) {
     case MUA_OK: return "ok";
     case MUA_ERR_ARG: return "argument out of range or NULL";
-    case MUA_ERR_UNSUPPORTED: return "unsupported configuration (bits != 4 or window too large)";
+    case MUA_ERR_UNSUPPORTED: return "unsupported configuration (bits != 4, window too large, odd tensor length or too many tensors)";
     case MUA_ERR_ALIGN: return "device pointer not 16-byte aligned";
     case MUA_ERR_CUDA: return "CUDA runtime error (see mua_last_cuda_error)";
     default: return "unknown error code";

@@ -1,4 +1,4 @@
-// Device-side building blocks of the two MicroAdam kernels (mua_select.cu,
+// Device-side building blocks of the two MicroAdam kernels (mua_select_warp.cu,
 // mua_apply.cu) and the argument block both take.
 //
 // [MicroAdam ¶n] is paragraph n of "MicroAdam (Sparse-Gradient Adaptive
@@ -28,8 +28,6 @@ constexpr int kChunks = kElemsPerThread / kChunk;
 constexpr int kMaxWindow = 64;            // m <= 64 (ages fit a 6-bit field)
 constexpr int kMaxSegments = 512;         // tensors of a list cut into blocks one by one
 constexpr int kMaxWindowEntries = 15360;  // m * row_stride per block, on chip
-constexpr int kCandCap = 2048;            // select: on-chip candidate list
-constexpr int kHistBins = 2048;           // radix digit of 11 bits
 constexpr uint32_t kEmptySlot = 0x0000FFFFu;  // I = -1, V = +0
 constexpr uint32_t kNil = 0xFFFFFFFFu;
 
@@ -37,9 +35,9 @@ constexpr uint32_t kNil = 0xFFFFFFFFu;
 constexpr int kHdrPair0 = 0;   // (-delta, Delta) for even t
 constexpr int kHdrPair1 = 2;   // (-delta, Delta) for odd t
 constexpr int kHdrStatus = 4;
+constexpr int kHdrBarrier = 5;  // arrivals at the fused kernel's grid barrier
 constexpr uint32_t kStatusNonFinite = 1u;
-constexpr uint32_t kStatusTimeout = 2u;   // a bounded wait gave up
-constexpr uint32_t kMaxWaitRounds = 1u << 22;  // try_wait rounds before giving up
+constexpr uint32_t kStatusTimeout = 2u;  // a bounded wait gave up
 
 struct Geometry {
   int64_t d;           // elements of this handle
@@ -55,7 +53,8 @@ struct Geometry {
 // One argument block for both kernels of step t.
 struct StepArgs {
   Geometry g;
-  float* params;
+  float* params;       // fp32 parameters, or NULL when params16 is used
+  uint16_t* params16;  // bf16 parameters (raw bits), or NULL
   const uint16_t* grads;
   uint8_t* codes;
   uint32_t* window;
@@ -69,8 +68,8 @@ struct StepArgs {
   uint32_t t_lo, t_hi;
   float lr, eps, decay, f1, f2;
   int32_t has_decay;
-  int32_t update_split;  // blocks with (j & 7) < update_split update in select
   uint32_t kp_recip;     // ceil(2^32 / kp): e / kp == __umulhi(e, kp_recip) for e < 2^16
+  uint64_t wait_ns;      // longest wait at a grid barrier before giving up
   float w1[kMaxWindow];  // fp32(beta1^r), r = age
   float w2[kMaxWindow];  // fp32(beta2^r)
   uint32_t keys[10][2];  // Philox round keys: seed + r*(W0, W1)
@@ -103,10 +102,6 @@ __device__ __forceinline__ void block_span(const StepArgs& A, int j, int64_t& st
   L = (int)min((int64_t)G.Bd, A.seg_len[lo] - off);
 }
 
-__device__ __forceinline__ bool update_in_select(const StepArgs& A, int j) {
-  return (j & 7) < A.update_split;
-}
-
 // ---------------------------------------------------------------- memory
 // A 4-byte load with a 64-byte L2 fetch-size hint: the update's sparse
 // parameter reads (a few per 128-byte line) then bring 64-byte halves from
@@ -115,6 +110,28 @@ __device__ __forceinline__ float ld_sparse_f32(const float* p) {
   float v;
   asm volatile("ld.global.L2::64B.f32 %0, [%1];" : "=f"(v) : "l"(p));
   return v;
+}
+__device__ __forceinline__ float ld_sparse_bf16(const uint16_t* p) {
+  uint16_t v;
+  asm volatile("ld.global.L2::64B.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return __uint_as_float((uint32_t)v << 16);
+}
+
+// Parameter storage: fp32, or bf16 rounded to nearest-even on every store.
+template <bool BF16>
+__device__ __forceinline__ float load_param_sparse(const StepArgs& A, int64_t i) {
+  if constexpr (BF16) return ld_sparse_bf16(A.params16 + i);
+  else return ld_sparse_f32(A.params + i);
+}
+template <bool BF16>
+__device__ __forceinline__ float load_param(const StepArgs& A, int64_t i) {
+  if constexpr (BF16) return __uint_as_float((uint32_t)A.params16[i] << 16);
+  else return A.params[i];
+}
+template <bool BF16>
+__device__ __forceinline__ void store_param(const StepArgs& A, int64_t i, float v) {
+  if constexpr (BF16) A.params16[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  else A.params[i] = v;
 }
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
@@ -128,6 +145,18 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
 }
+// A 4-byte load of data this kernel also writes (the apply kernel's codes,
+// which it overwrites in place): not through the read-only path.
+__device__ __forceinline__ uint32_t ld_rw_u32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// 32-bit shared-window address of a shared-memory object.
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
 
 template <int T>
 __device__ __forceinline__ int elem_index(int c, int tid, int e) {
@@ -137,7 +166,9 @@ __device__ __forceinline__ int elem_index(int c, int tid, int e) {
 // Loads the thread's 4 chunks: gradient bits as 4 words per chunk (word w holds
 // elements 2w (low half) and 2w+1 (high half)), codes as one word per chunk
 // (nibble e = element e). Elements at or past L read as g = +0, code = 0.
-template <int T, bool VEC>
+// The codes are read with coherent loads: the caller overwrites them.
+// FULL (with VEC): all 32 T elements lie inside the block, no checks.
+template <int T, bool VEC, bool FULL = false>
 __device__ __forceinline__ void load_block(const uint16_t* __restrict__ grads,
                                            const uint8_t* __restrict__ codes, int64_t start,
                                            int L, int tid, uint4 (&gv)[kChunks],
@@ -145,9 +176,9 @@ __device__ __forceinline__ void load_block(const uint16_t* __restrict__ grads,
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
     const int e0 = elem_index<T>(c, tid, 0);
-    if (VEC && e0 + kChunk <= L) {
+    if ((VEC && FULL) || (VEC && e0 + kChunk <= L)) {
       gv[c] = ld_stream_v4(grads + start + e0);
-      cv[c] = ld_stream_u32(codes + ((start + e0) >> 1));
+      cv[c] = ld_rw_u32(codes + ((start + e0) >> 1));
     } else {
       uint32_t w[4] = {0u, 0u, 0u, 0u};
       uint32_t cw = 0u;
@@ -218,21 +249,6 @@ __device__ __forceinline__ void fill_levels(float* lv, float delta, float unit) 
   }
 }
 
-// a = f32(g) + Q^{-1}(code) for every element of the thread (stage (1)).
-__device__ __forceinline__ void dequant_block(const uint4 (&gv)[kChunks],
-                                              const uint32_t (&cv)[kChunks], const float* lv,
-                                              uint32_t (&ab)[kElemsPerThread]) {
-#pragma unroll
-  for (int c = 0; c < kChunks; ++c) {
-#pragma unroll
-    for (int e = 0; e < kChunk; ++e) {
-      const float gf = __uint_as_float(grad_bits(gv[c], e));
-      const float lev = lv[(cv[c] >> (4 * e)) & 0xFu];
-      ab[c * kChunk + e] = __float_as_uint(__fadd_rn(gf, lev));
-    }
-  }
-}
-
 // One 4-bit code of stage (4): c = min(15, floor((floor(2^16 s) + r) / 2^16)),
 // s16 = 2^16 s >= 0, r a 16-bit draw. Returns the code in bits 16..19 of the
 // result (bits 0..15 are scratch); the caller shifts it into place.
@@ -241,99 +257,40 @@ __device__ __forceinline__ uint32_t quantize_code_hi(float s16, uint32_t r) {
   return __viaddmin_u32(big, r, 0x4B0FFFFFu);  // min(big + r, code 15)
 }
 
-// ---------------------------------------------------------------- TMA bulk copies
-// 1-D bulk copies global -> shared (cp.async.bulk, no multicast) completing
-// on an mbarrier with a transaction count. Waits are bounded: after
-// kMaxWaitRounds unsuccessful try_wait rounds the caller gets false.
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
-}
-__device__ __forceinline__ void mbar_init_fence() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-               ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n"
-      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}"
-      : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
-  return ok != 0u;
-}
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kMaxWaitRounds; ++it)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
-}
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
-                                         uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
-}
-// Orders this thread's earlier generic-proxy shared-memory accesses before
-// later async-proxy (bulk copy) accesses.
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// The thread's 4 chunks of a block staged in shared memory (gradients as bf16
-// at g, codes at c; both start at the block's first element).
-template <int T>
-__device__ __forceinline__ void load_block_smem(const uint16_t* g, const uint8_t* c, int tid,
-                                                uint4 (&gv)[kChunks], uint32_t (&cv)[kChunks]) {
+// Stage (4) for the 8 elements of a chunk [MicroAdam ¶1]: a2[i] holds the
+// pair (a of element 2i, a of element 2i + 1) as fp32 bits (low, high);
+// elements whose bit is set in `selbits` were selected and quantize as +0;
+// x is the chunk's Philox4x32-10 output (element e draws the (e mod 2)-th
+// 16-bit half of word e / 2); dn2 and inv2 hold (delta, delta) and
+// (2^16 * 15 / (Delta - delta)) twice. Returns the 8 codes packed into one
+// word, element e in bits 4e .. 4e + 3.
+//   s16 = (a - delta) * inv16, big = 2^23 + s16 rounded toward zero, so the low
+//   mantissa of big is floor(s16); the code is min(15, (floor(s16) + r) >> 16),
+//   which sits in bits 16..19 of min(big + r, 0x4B0FFFFF), i.e. in byte 2.
+__device__ __forceinline__ uint32_t quantize8(const uint64_t (&a2)[4], uint32_t selbits,
+                                              const uint4& x, uint64_t dn2, uint64_t inv2) {
+  const uint64_t magic2 = f2_pack(8388608.0f, 8388608.0f);
+  uint32_t hi[kChunk];
 #pragma unroll
-  for (int k = 0; k < kChunks; ++k) {
-    const int e0 = elem_index<T>(k, tid, 0);
-    gv[k] = *reinterpret_cast<const uint4*>(g + e0);
-    cv[k] = *reinterpret_cast<const uint32_t*>(c + (e0 >> 1));
+  for (int i = 0; i < 4; ++i) {
+    uint64_t a = a2[i];
+    if ((selbits >> (2 * i)) & 1u) a &= 0xFFFFFFFF00000000ull;  // selected: a = +0
+    if ((selbits >> (2 * i + 1)) & 1u) a &= 0x00000000FFFFFFFFull;
+    const uint64_t big2 = f2_add_rz(f2_mul_rn(f2_sub_rn(a, dn2), inv2), magic2);
+    const uint32_t xw = chunk_word(x, i);
+    hi[2 * i] = __viaddmin_u32((uint32_t)big2, xw & 0xFFFFu, 0x4B0FFFFFu);
+    hi[2 * i + 1] = __viaddmin_u32((uint32_t)(big2 >> 32), xw >> 16, 0x4B0FFFFFu);
   }
+  // Byte 2 of each (0..15, the code): even elements into one word, odd ones
+  // into another, then one nibble interleave.
+  const uint32_t ev = __byte_perm(__byte_perm(hi[0], hi[2], 0x0062u),
+                                  __byte_perm(hi[4], hi[6], 0x0062u), 0x5410u);
+  const uint32_t od = __byte_perm(__byte_perm(hi[1], hi[3], 0x0062u),
+                                  __byte_perm(hi[5], hi[7], 0x0062u), 0x5410u);
+  return ev | (od << 4);
 }
 
 // ---------------------------------------------------------------- scans
-// Inclusive block scan over T threads (T a multiple of 32). `scratch` needs
-// T/32 entries. Ends with a barrier so scratch can be reused at once.
-template <int T, typename V>
-__device__ __forceinline__ V block_inclusive_scan(V x, V* scratch, V& total) {
-  constexpr int NW = T / 32;
-  const int lane = threadIdx.x & 31;
-  const int wid = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const V y = __shfl_up_sync(0xFFFFFFFFu, x, o);
-    if (lane >= o) x += y;
-  }
-  if constexpr (NW == 1) {
-    total = __shfl_sync(0xFFFFFFFFu, x, 31);
-    return x;
-  } else {
-    if (lane == 31) scratch[wid] = x;
-    __syncthreads();
-    if (wid == 0) {
-      V w = (lane < NW) ? scratch[lane] : V(0);
-#pragma unroll
-      for (int o = 1; o < NW; o <<= 1) {
-        const V y = __shfl_up_sync(0xFFFFFFFFu, w, o);
-        if (lane >= o) w += y;
-      }
-      if (lane < NW) scratch[lane] = w;
-    }
-    __syncthreads();
-    const V off = (wid > 0) ? scratch[wid - 1] : V(0);
-    total = scratch[NW - 1];
-    __syncthreads();
-    return x + off;
-  }
-}
-
 // Inclusive block scan with a single barrier: every warp re-scans the warp
 // totals itself. `scratch` (T/32 entries) must not be written again before
 // the next barrier.
@@ -362,25 +319,6 @@ __device__ __forceinline__ V block_scan_1bar(V x, V* scratch, V& total) {
     const V off = __shfl_sync(0xFFFFFFFFu, w, (wid + 31) & 31);
     total = __shfl_sync(0xFFFFFFFFu, w, NW - 1);
     return x + (wid > 0 ? off : V(0));
-  }
-}
-
-// Block max of a uint32 (ends with a barrier).
-template <int T>
-__device__ __forceinline__ uint32_t block_max_u32(uint32_t x, uint32_t* scratch) {
-  constexpr int NW = T / 32;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = max(x, __shfl_xor_sync(0xFFFFFFFFu, x, o));
-  if constexpr (NW == 1) {
-    return x;
-  } else {
-    if ((threadIdx.x & 31) == 0) scratch[threadIdx.x >> 5] = x;
-    __syncthreads();
-    uint32_t r = scratch[0];
-#pragma unroll
-    for (int w = 1; w < NW; ++w) r = max(r, scratch[w]);
-    __syncthreads();
-    return r;
   }
 }
 
@@ -438,14 +376,16 @@ __host__ __device__ inline uint32_t update_smem_bytes(int threads, int Bd, int k
 
 // Stage (6) for block j [MicroAdam ¶1]: m_hat = AdamStats(beta1, G) and
 // v_hat = AdamStats(beta2, G^2) over the block's window rows, then
-// p <- p*(1 - lr*wd) (dense, if wd != 0) and p <- p - lr*m_hat/(eps + sqrt(v_hat))
-// on the window's index union. The rows are staged in shared memory and a
+// p <- p*(1 - lr*wd) - lr*m_hat/(eps + sqrt(v_hat)) on the window's index union
+// and, if wd != 0, p <- p*(1 - lr*wd) on every other parameter of the block:
+// each parameter is read and written once, and a bf16 parameter (BF16) is
+// rounded once. The rows are staged in shared memory and a
 // bitmask + popcount prefix gives each index its union rank. The sums run one
 // row at a time, oldest row first: the indices of one row are distinct, so no
 // two threads touch one accumulator within a row, and every accumulator sees
 // its terms in the same order on every run. Called by all T threads, after a
 // barrier.
-template <int T>
+template <int T, bool BF16>
 __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t start, int L,
                                              uint8_t* smem, const float* s_w1,
                                              const float* s_w2) {
@@ -528,9 +468,10 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
     uidx[rank] = (uint16_t)idx;
     acc[rank] = make_float2(0.0f, 0.0f);
   }
-  if (A.has_decay) {
-    float* pb = A.params + start;
-    for (int i = tid; i < L; i += T) pb[i] = __fmul_rn(pb[i], A.decay);
+  if (A.has_decay) {  // decay alone off the union (the union's comes with its update)
+    for (int i = tid; i < L; i += T)
+      if (!((mask[i >> 5] >> (i & 31)) & 1u))
+        store_param<BF16>(A, start + i, __fmul_rn(load_param<BF16>(A, start + i), A.decay));
   }
   __syncthreads();
 
@@ -569,13 +510,14 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
       const float2 z = acc[r];
       mh[b] = __fmul_rn(A.f1, z.x);
       vh[b] = __fmul_rn(A.f2, z.y);
-      pv[b] = ld_sparse_f32(A.params + start + idx[b]);
+      pv[b] = load_param_sparse<BF16>(A, start + idx[b]);
+      if (A.has_decay) pv[b] = __fmul_rn(pv[b], A.decay);
     }
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
       if (idx[b] == kNil) continue;
       const float u = __fmul_rn(mh[b], rcp_approx(__fadd_rn(A.eps, sqrt_approx(vh[b]))));
-      A.params[start + idx[b]] = __fsub_rn(pv[b], __fmul_rn(A.lr, u));
+      store_param<BF16>(A, start + idx[b], __fsub_rn(pv[b], __fmul_rn(A.lr, u)));
       if (A.mhat) {
         A.mhat[start + idx[b]] = mh[b];
         A.vhat[start + idx[b]] = vh[b];
@@ -595,14 +537,33 @@ __device__ __forceinline__ void load_weights(const StepArgs& A, float* s_w1, flo
 }
 
 // ---------------------------------------------------------------- launchers
+constexpr int kMaxDevices = 64;
+
+// Raises a kernel's dynamic shared-memory limit to at least `smem` bytes, once
+// per device and size: `opted` is the caller's record for that kernel (one
+// static array per kernel instance). Devices past kMaxDevices opt in on every
+// call.
+template <typename Kern>
+cudaError_t opt_in_smem(Kern kern, uint32_t smem, uint32_t (&opted)[kMaxDevices]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool known = dev >= 0 && dev < kMaxDevices;
+  if (known && opted[dev] >= smem) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess && known) opted[dev] = smem;
+  return e;
+}
+
 // Host-side launchers (defined next to their kernels). Return a cudaError_t.
-cudaError_t launch_select(const StepArgs& args, int threads, bool vec, bool persistent,
-                          uint32_t smem, cudaStream_t stream);
 cudaError_t launch_apply(const StepArgs& args, int threads, bool vec, uint32_t smem,
-                         cudaStream_t stream);
-uint32_t select_smem_bytes(int threads, int Bd, int kp, int m);
+                         cudaStream_t stream);  // bf16 parameters when args.params16
 cudaError_t launch_select_warp(const StepArgs& args, bool vec, cudaStream_t stream);
 uint32_t select_warp_smem_bytes(int Bd);
 uint32_t apply_smem_bytes(int threads, int Bd, int kp, int m);
+// The fused one-launch step (mua_fused.cu): how many of its CTAs the current
+// device holds at once (0 if it cannot run this geometry), and its launch.
+int fused_max_blocks(int Bd, int kp, int m, bool vec, bool bf16);
+cudaError_t launch_fused(const StepArgs& args, bool vec, cudaStream_t stream);
 
 }  // namespace mua

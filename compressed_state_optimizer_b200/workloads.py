@@ -67,6 +67,7 @@ class Workload:
     wd: float = 0.0
     seed: int = 0x5EED0000
     per_tensor: bool = False       # blocks cut per tensor of ``shapes`` (else over the flat vector)
+    params: str = "f32"            # parameter storage: "f32" | "bf16"
 
     def segments(self):
         """Tensor lengths when blocks are cut per tensor, else None."""

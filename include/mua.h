@@ -46,8 +46,9 @@ extern "C" {
 
 /* Status bits (sticky, in the state header). */
 #define MUA_STATUS_NONFINITE 1u  /* some a_t was NaN or +-inf; results unspecified  */
-#define MUA_STATUS_TIMEOUT 2u    /* a kernel's bounded wait for its own bulk copy gave
-                                    up; that step's results are unspecified           */
+#define MUA_STATUS_TIMEOUT 2u    /* a CTA of the fused step gave up waiting at its grid
+                                    barrier (see mua_set_wait_limit_ns); that step's
+                                    results are unspecified                           */
 
 /* Fields written by mua_state_layout(). */
 #define MUA_LAYOUT_HEADER 0      /* byte offset of the 256-byte scalar header        */
@@ -103,9 +104,8 @@ int mua_create_shard(int64_t d_total, int32_t block_size, int32_t k_per_block,
  * Errors: MUA_ERR_ARG for NULL pointers, n_seg < 1, a length < 1 or the
  * arguments mua_create rejects; MUA_ERR_UNSUPPORTED for an odd length (a
  * block must start on a byte of the 4-bit codes), n_seg > MUA_MAX_SEGMENTS,
- * and what mua_create cannot hold. Variant 2 of mua_set_select_variant is not
- * available for these handles. The 16-byte vector path is used when B_d and
- * every length are multiples of 8.
+ * and what mua_create cannot hold. The 16-byte vector path is used when B_d
+ * and every length are multiples of 8.
  */
 #define MUA_MAX_SEGMENTS 512
 int mua_create_segmented(const int64_t* seg_len, int32_t n_seg, int32_t block_size,
@@ -130,19 +130,26 @@ int64_t mua_state_bytes(mua_t h);
  * (low half; 0xFFFF = empty slot) | bf16 V << 16; row (t mod m) of block j
  * holds the block's Top-k of step t in ascending index order. The header
  * holds two (-delta, Delta) fp32 pairs at words 0-1 and 2-3 (pair t mod 2 is
- * step t's (delta_t, Delta_t)) and the status word at word 4.
+ * step t's (delta_t, Delta_t)), the status word at word 4 and the fused step's
+ * barrier count at word 5 (reset by every fused step).
  */
 int mua_state_layout(mua_t h, int64_t* out);
 
 /*
- * mua_step — one full MicroAdam step t [MicroAdam ¶1] on `stream`:
- * mua_select followed by mua_apply, without statistics outputs.
+ * mua_step — one full MicroAdam step t [MicroAdam ¶1] on `stream`.
+ * For a whole vector (not a shard) of blocks of at most 16384 entries whose
+ * CTAs the current device can all hold at once (up to one block per SM), the
+ * step is ONE cooperative launch that keeps a_t in registers across a
+ * grid-wide barrier (bounded: see mua_set_wait_limit_ns); otherwise it is
+ * mua_select followed by mua_apply. Both give the same bytes.
+ * mua_step_launches tells which applies.
  *   params  device, fp32[d], updated in place
  *   grads   device, bf16[d] (raw 16-bit patterns), read only
  *   state   device, mua_state_bytes(h) bytes, updated in place
- *   lr, beta1, beta2, eps, wd   fp32 hyper-parameters; 0 <= beta < 1,
- *           eps >= 0, all finite; wd is decoupled weight decay applied to
- *           every parameter as p *= (1 - lr*wd) before the update
+ *   lr, beta1, beta2, eps, wd   fp32 hyper-parameters, all finite;
+ *           0 <= beta < 1; eps > 0 (an index whose window values are all
+ *           zero would otherwise divide 0 by 0); wd is decoupled weight decay
+ *           applied to every parameter as p *= (1 - lr*wd) before the update
  *   t       step number: 1 for the first step, then t+1 on every call
  *   seed    key of the Philox4x32-10 stream of the stochastic rounding
  * Errors: MUA_ERR_ARG (NULL pointer, t < 1, bad hyper-parameter),
@@ -153,14 +160,29 @@ int mua_step(mua_t h, float* params, const uint16_t* grads, void* state, float l
              void* stream);
 
 /*
+ * mua_step_bf16 — mua_step for bf16 parameters: params is bf16[d] (raw
+ * 16-bit patterns, device, 16-byte aligned), updated in place; there is no
+ * fp32 copy. Every parameter the step changes (the window's index union, and
+ * with wd != 0 every parameter) is computed in fp32 from its bf16 value and
+ * rounded once to bf16, to nearest with ties to even: the page's full
+ * fine-tune of LLaMA-2 7B on a single 40 GB GPU [MicroAdam ¶4] leaves no room
+ * for 27 GB of fp32 parameters. Everything else (state, window, codes) is that
+ * of mua_step. Arguments and errors as mua_step.
+ */
+int mua_step_bf16(mua_t h, uint16_t* params, const uint16_t* grads, void* state, float lr,
+                  float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+                  void* stream);
+
+/*
  * mua_select — first half of step t [MicroAdam ¶1]: stages (1)-(3) and (5):
  * a_t from grads and e_t, the per-block Top-k written to row t mod m of G,
- * the per-block residual min/max folded into the (-delta_{t+1}, Delta_{t+1})
- * pair of the header (reset first, see mua_minmax_offset), and stage (6), the
- * AdamStats update of params, for the blocks this kernel owns (see
- * mua_set_update_split). Arguments as mua_step; mhat / vhat as mua_apply.
+ * and the per-block residual min/max folded into the (-delta_{t+1},
+ * Delta_{t+1}) pair of the header (reset first, see mua_minmax_offset).
+ * params, mhat and vhat are not touched: params may be NULL (for bf16
+ * parameters pass NULL); non-NULL pointers are checked for alignment.
  * mua_select(t) and mua_apply(t) must be called in that order with identical
  * arguments; a sharded caller all-reduces the header pair between them.
+ * Arguments and errors as mua_step.
  */
 int mua_select(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
                float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
@@ -177,48 +199,49 @@ int64_t mua_minmax_offset(mua_t h, int64_t t);
 /*
  * mua_apply — second half of step t after mua_select(t): stage (4), the
  * quantization of the residual into e_{t+1} with (delta_{t+1}, Delta_{t+1}),
- * and stage (6) for the blocks mua_select left. If mhat / vhat are non-NULL
- * (device, fp32[d]), m_hat and v_hat are also written at every index of the
- * window's union (other entries are left untouched) by whichever of the two
- * calls updates that block, for testing and diagnostics. Arguments and errors
- * as mua_step.
+ * and stage (6), the AdamStats update of the parameters. If mhat / vhat are
+ * non-NULL (device, fp32[d]), m_hat and v_hat are also written at every index
+ * of the window's union (other entries are left untouched), for testing and
+ * diagnostics. Arguments and errors as mua_step.
  */
 int mua_apply(mua_t h, float* params, const uint16_t* grads, void* state, float lr,
               float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
               float* mhat, float* vhat, void* stream);
 
 /*
- * mua_set_update_split — which kernel applies stage (6) to block j: mua_select
- * when (j mod 8) < split, mua_apply otherwise; 0 <= split <= 8 (default 4).
- * Only the CTA shapes of mua_select (variants 1, 2) use it: with the default
- * warp-per-block select every block is updated in mua_apply.
- * The results do not depend on it (each block is updated exactly once, by
- * the same arithmetic); it only moves HBM traffic between the two kernels to
- * balance them. Host only; MUA_ERR_ARG when out of range.
+ * mua_apply_bf16 — mua_apply for bf16 parameters (see mua_step_bf16).
  */
-int mua_set_update_split(mua_t h, int32_t split);
+int mua_apply_bf16(mua_t h, uint16_t* params, const uint16_t* grads, void* state, float lr,
+                   float beta1, float beta2, float eps, float wd, int64_t t, uint64_t seed,
+                   float* mhat, float* vhat, void* stream);
 
 /*
- * mua_set_select_variant — the kernel shape of mua_select (results are
- * identical for every variant):
- *   0 (default) one warp per block, many blocks in flight per SM; all
- *     parameter updates then run in mua_apply (mua_set_update_split ignored);
- *   1 one CTA per block;
- *   2 persistent CTAs streaming each next block into shared memory with
- *     bulk copies (needs B_d % 32 == 0, at least 2 blocks and a flat cut,
- *     else MUA_ERR_UNSUPPORTED).
- * Variants 1 and 2 also return MUA_ERR_UNSUPPORTED when one block's select
- * and AdamStats working set does not fit one CTA's shared memory.
- * Host only; MUA_ERR_ARG for other values.
+ * mua_step_launches — kernel launches mua_step(h, ...) (bf16_params == 0) or
+ * mua_step_bf16(h, ...) (bf16_params != 0) makes on the current device: 1
+ * (the fused one-launch step) or 2 (mua_select + mua_apply). Queries the
+ * device once per device, handle and parameter type. Returns MUA_ERR_ARG for
+ * a NULL handle, MUA_ERR_CUDA if the query fails.
  */
-int mua_set_select_variant(mua_t h, int32_t variant);
+int mua_step_launches(mua_t h, int32_t bf16_params);
+
+/*
+ * mua_set_wait_limit_ns — bound, in nanoseconds of the GPU's global timer, on
+ * how long a CTA of the fused step waits at its grid barrier before it sets
+ * MUA_STATUS_TIMEOUT and returns without finishing the step (default 2 s,
+ * far above a step's duration; the CTAs of a cooperative launch are all
+ * resident, so the wait normally ends in microseconds). A limit <= 0 makes a
+ * CTA give up as soon as it would wait: a way to exercise that path in tests.
+ * Host only; MUA_ERR_ARG for a NULL handle.
+ */
+int mua_set_wait_limit_ns(mua_t h, int64_t ns);
 
 /*
  * mua_get_status — copy the state's sticky status word (MUA_STATUS_* bits)
- * into the host integer *out. Synchronizes `stream`. Returns MUA_ERR_CUDA if
- * the copy fails.
+ * into the host integer *out, after the work already enqueued on `stream`.
+ * Synchronizes `stream`. Returns MUA_ERR_ARG for NULL arguments and
+ * MUA_ERR_CUDA if the copy fails.
  */
-int mua_get_status(mua_t h, const void* state, uint32_t* out, void* stream);
+int mua_get_status(mua_t h, const void* state, void* stream, int32_t* out);
 
 /* mua_strerror — static text for a return code. */
 const char* mua_strerror(int code);

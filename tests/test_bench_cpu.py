@@ -20,7 +20,7 @@ def test_reference_arm_json_line(oracle_lib):
     assert d["impl"] == "reference" and d["unit"] == "Gparams/s" and d["value"] > 0
     assert d["higher_is_better"] is True and d["steps"] == 2 and d["warmup"] == 1
     assert d["n_gpus"] == 1 and d["config"]["workload"] == "flat_d2^20_normal"
-    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == os.cpu_count()
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
 
 
@@ -34,3 +34,5 @@ def test_workload_names():
     w = bench.get_workload("llama2_7b_per_tensor", wd=0.1)
     assert w.wd == 0.1 and len(w.segments()) == 291 and sum(w.segments()) == w.d
     assert bench.get_workload("llama2_7b").segments() is None
+    assert bench.get_workload("llama2_7b_bf16").params == "bf16"
+    assert bench.get_workload("llama2_7b").params == "f32"

@@ -63,15 +63,11 @@ def compare_stats(mhat, vhat, stats, what=""):
 
 def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0.9,
                b2=0.999, eps=1e-8, wd=0.0, grads_fn=None, stats=True, use_step=False,
-               split=None, variant=None, segments=None):
+               segments=None):
     torch, MicroAdam, workloads = _mods()
     w = workloads.Workload("parity", d, Bd, kb, m, kind, steps, seed=seed)
     p0 = workloads.make_params(d, seed=7)
     mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m, segments=segments)
-    if variant is not None:
-        mo.set_select_variant(variant)
-    if split is not None:
-        mo.set_update_split(split)
     state = mo.new_state("cuda")
     p_gpu = p0.cuda()
     ost = oracle.new_state(d, Bd, kb, m, segments=segments)
@@ -98,12 +94,9 @@ def run_parity(d, Bd, kb, m, steps, *, kind="normal", seed=0x1234, lr=1e-3, b1=0
     return mo, state, p_gpu
 
 
-@pytest.mark.parametrize("variant,split", [(0, 0), (1, 4), (1, 0), (1, 8), (2, 4)])
-def test_flat_2p20_twenty_steps(variant, split):
-    """d = 2^20, N(0,1) bf16 gradients, B_d = 16384, k_b = 164, m = 10, 20 steps,
-    for every select kernel shape (warp per block, CTA per block, persistent
-    CTAs) and with the parameter update in either kernel or shared."""
-    run_parity(1 << 20, 16384, 164, 10, 20, split=split, variant=variant)
+def test_flat_2p20_twenty_steps():
+    """d = 2^20, N(0,1) bf16 gradients, B_d = 16384, k_b = 164, m = 10, 20 steps."""
+    run_parity(1 << 20, 16384, 164, 10, 20)
 
 
 def test_flat_2p20_through_mua_step():
@@ -128,15 +121,8 @@ def test_shapes(d, Bd, kb, m, steps, kind):
     run_parity(d, Bd, kb, m, steps, kind=kind)
 
 
-@pytest.mark.parametrize("variant,split", [(0, 0), (1, 4), (1, 8)])
-def test_weight_decay(variant, split):
-    run_parity(9 * 4096 + 100, 4096, 41, 5, 6, wd=0.1, lr=1e-2, split=split, variant=variant)
-
-
-@pytest.mark.parametrize("variant", [1, 2])
-def test_shapes_other_variants(variant):
-    """Ragged blocks and ties through the CTA-per-block and persistent shapes."""
-    run_parity(5 * 2048 + 777, 2048, 21, 3, 8, kind="t3", variant=variant, split=4)
+def test_weight_decay():
+    run_parity(9 * 4096 + 100, 4096, 41, 5, 6, wd=0.1, lr=1e-2)
 
 
 def test_ties_and_zero_blocks():
@@ -152,6 +138,146 @@ def test_ties_and_zero_blocks():
         return workloads.grads_from_values(x)
 
     run_parity(d, Bd, 11, 4, 8, grads_fn=grads)
+
+
+def test_one_signed_blocks():
+    """Blocks whose values lie on one side of zero (all positive, all negative)
+    beside mixed ones. The select kernel takes a block's residual min and max
+    from the candidates it did not select when they reach past every lane's
+    threshold; in a one-signed block one side does not, and its extra pass over
+    the block's unselected elements decides it."""
+    torch, _, workloads = _mods()
+    Bd = 16384
+    d = 6 * Bd + 4000
+    rng = np.random.default_rng(5)
+
+    def grads(t):
+        x = np.abs(rng.standard_normal(d)).astype(np.float32)
+        x[Bd:2 * Bd] *= -1.0                            # all negative
+        x[3 * Bd:4 * Bd] = rng.standard_normal(Bd)      # mixed
+        x[5 * Bd:] *= 1e-3                              # small, positive, ragged tail
+        return workloads.grads_from_values(x)
+
+    run_parity(d, Bd, 164, 4, 6, grads_fn=grads)
+
+
+@pytest.mark.parametrize("d,Bd,kb,m,steps,kind,wd", [
+    (1 << 20, 16384, 164, 10, 20, "normal", 0.0),      # the 2^20 vector, 20 steps
+    (5 * 2048 + 777, 2048, 21, 3, 8, "t3", 0.0),       # ragged odd-length last block
+    (4 * 1022 + 301, 1022, 11, 4, 8, "normal", 0.0),   # B_d % 8 != 0: scalar path
+    (9 * 4096 + 100, 4096, 41, 5, 6, "t3", 0.1),       # weight decay
+    (3 * 16384, 16384, 164, 37, 40, "normal", 0.0),    # m = 37
+])
+def test_fused_step(d, Bd, kb, m, steps, kind, wd):
+    """mua_step as ONE launch (blocks fit the device at once) against the oracle,
+    every step."""
+    torch, MicroAdam, _ = _mods()
+    assert MicroAdam(d, block_size=Bd, k_per_block=kb, window=m).step_launches() == 1
+    run_parity(d, Bd, kb, m, steps, kind=kind, use_step=True, wd=wd,
+               lr=1e-2 if wd else 1e-3)
+
+
+def test_fused_equals_two_kernels():
+    """The fused step and select + apply give the same bytes, step after step."""
+    torch, MicroAdam, workloads = _mods()
+    d, Bd, kb, m = 7 * 16384 + 4000, 16384, 164, 5
+    w = workloads.Workload("pair", d, Bd, kb, m, "t3", 12, seed=4)
+    hyper = dict(lr=1e-3, beta1=.9, beta2=.999, eps=1e-8, wd=0., seed=21)
+    mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m)
+    assert mo.step_launches() == 1
+    sa, sb = mo.new_state(), mo.new_state()
+    pa = workloads.make_params(d).cuda()
+    pb = pa.clone()
+    for t in range(1, 13):
+        g = workloads.make_grads(w, t).cuda()
+        mo.step(pa, g, sa, t=t, **hyper)
+        mo.select(pb, g, sb, t=t, **hyper)
+        mo.apply(pb, g, sb, t=t, **hyper)
+        torch.cuda.synchronize()
+        assert torch.equal(sa[:20], sb[:20]) and torch.equal(sa[32:], sb[32:]), t
+        assert torch.equal(pa, pb), t
+
+
+def test_fused_barrier_timeout_sets_status():
+    """A CTA that waits longer than the limit at the fused step's grid barrier
+    sets MUA_STATUS_TIMEOUT and returns; the kernel ends, the context stays
+    usable and a fresh state then steps normally."""
+    torch, MicroAdam, workloads = _mods()
+    from compressed_state_optimizer_b200.binding import MUA_STATUS_TIMEOUT
+    d, Bd, kb, m = 32 * 16384, 16384, 164, 4
+    w = workloads.Workload("timeout", d, Bd, kb, m, "normal", 5, seed=6)
+    hyper = dict(lr=1e-3, beta1=.9, beta2=.999, eps=1e-8, wd=0., seed=3)
+    mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m)
+    assert mo.step_launches() == 1
+    mo.set_wait_limit_ns(0)  # give up at once
+    state = mo.new_state()
+    p = workloads.make_params(d).cuda()
+    for t in range(1, 6):
+        mo.step(p, workloads.make_grads(w, t).cuda(), state, t=t, **hyper)
+    torch.cuda.synchronize()
+    assert mo.status(state) & MUA_STATUS_TIMEOUT
+    mo.set_wait_limit_ns(2_000_000_000)
+    run_parity(d, Bd, kb, m, 3, use_step=True)
+
+
+def run_parity_bf16(d, Bd, kb, m, steps, *, kind="t3", seed=0x77, lr=1e-3, wd=0.0,
+                    use_step=True, segments=None):
+    """bf16 parameters against the oracle's bf16-parameter step. Each step the
+    oracle starts from the GPU's parameters; the window rows, codes and
+    delta/Delta must agree bit for bit. The kernel forms each new parameter in
+    fp32, the oracle in fp64, so the GPU's bf16 value must lie within half a
+    bf16 step of the oracle's exact value plus the fp32 tolerance of the fp32
+    tests, 1e-5 * max(|exact|, lr): away from cancellation that admits the
+    nearest-even value only, or its neighbour where the exact value is within
+    1e-5 of a rounding midpoint; where p*(1 - lr*wd) and lr*u nearly cancel,
+    the fp32 rounding of the two terms (about 1e-9 at lr = 1e-2) can exceed a
+    bf16 step of the tiny result, and the absolute floor admits that."""
+    torch, MicroAdam, workloads = _mods()
+    w = workloads.Workload("bf16", d, Bd, kb, m, kind, steps, seed=seed)
+    mo = MicroAdam(d, block_size=Bd, k_per_block=kb, window=m, segments=segments)
+    state = mo.new_state("cuda")
+    p_gpu = workloads.make_params(d, seed=7).to(torch.bfloat16).cuda()
+    ost = oracle.new_state(d, Bd, kb, m, segments=segments)
+    hyper = dict(lr=lr, beta1=0.9, beta2=0.999, eps=1e-8, wd=wd)
+    exact = np.zeros(d, dtype=np.float64)
+    changed = 0
+    for t in range(1, steps + 1):
+        g = workloads.make_grads(w, t)
+        p_ref = workloads.bf16_bits(p_gpu)
+        before = p_ref.copy()
+        if use_step:
+            mo.step(p_gpu, g.cuda(), state, t=t, seed=seed, **hyper)
+        else:
+            mo.select(p_gpu, g.cuda(), state, t=t, seed=seed, **hyper)
+            mo.apply(p_gpu, g.cuda(), state, t=t, seed=seed, **hyper)
+        oracle.step(ost, p_ref, workloads.bf16_bits(g), t=t, seed=seed, p_exact=exact, **hyper)
+        torch.cuda.synchronize()
+        compare_state(mo, state, ost, t, d, m, kb, f"(bf16 params d={d})")
+        got = workloads.bf16_bits(p_gpu)
+        gf = (got.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        nxt = ((got.astype(np.uint32) + 1) << 16).view(np.float32).astype(np.float64)
+        half_ulp = np.abs(nxt - gf) / 2
+        bound = half_ulp + RTOL * np.maximum(np.abs(exact), lr)
+        bad = np.flatnonzero(np.abs(gf - exact) > bound)
+        assert bad.size == 0, (t, bad[:5], got[bad[:5]], p_ref[bad[:5]], exact[bad[:5]])
+        changed += int(np.count_nonzero(got != before))
+    assert changed > 0
+
+
+@pytest.mark.parametrize("d,Bd,kb,m,steps,kind,wd,use_step", [
+    (1 << 20, 16384, 164, 10, 12, "normal", 0.0, True),     # fused one-launch step
+    (1 << 20, 16384, 164, 10, 8, "t3", 0.1, False),         # select + apply, weight decay
+    (5 * 2048 + 777, 2048, 21, 3, 6, "t3", 0.05, True),     # ragged
+    (4 * 1022 + 302, 1022, 11, 4, 6, "normal", 0.0, False),  # B_d % 8 != 0: scalar path
+])
+def test_bf16_params(d, Bd, kb, m, steps, kind, wd, use_step):
+    run_parity_bf16(d, Bd, kb, m, steps, kind=kind, wd=wd, use_step=use_step,
+                    lr=1e-2 if wd else 1e-3)
+
+
+def test_bf16_params_segmented():
+    segs = [3 * 4096 + 64, 512, 4096]
+    run_parity_bf16(sum(segs), 4096, 41, 5, 6, segments=segs, wd=0.05, lr=1e-2)
 
 
 def test_adam_reduction_on_gpu():
@@ -241,19 +367,18 @@ def test_select_paths(kb):
 
 
 SEGMENTED = [
-    # (B_d, k_b, m, steps, tensor lengths, kind, select variant)
-    (16384, 164, 4, 8, [2 * 16384 + 1000, 8000, 16384, 4096 + 8, 30000], "t3", None),
-    (16384, 164, 4, 6, [2 * 16384 + 1000, 8000, 16384, 4096 + 8, 30000], "t3", 1),
-    (2048, 21, 3, 6, [5000, 2, 2048, 3070, 6], "normal", None),  # lengths not all 8k: scalar path
-    (8192, 82, 10, 12, [8192 * 3, 4104, 9000, 1000], "t3", None),
+    # (B_d, k_b, m, steps, tensor lengths, kind)
+    (16384, 164, 4, 8, [2 * 16384 + 1000, 8000, 16384, 4096 + 8, 30000], "t3"),
+    (2048, 21, 3, 6, [5000, 2, 2048, 3070, 6], "normal"),  # lengths not all 8k: scalar path
+    (8192, 82, 10, 12, [8192 * 3, 4104, 9000, 1000], "t3"),
 ]
 
 
-@pytest.mark.parametrize("Bd,kb,m,steps,segs,kind,variant", SEGMENTED)
-def test_segmented(Bd, kb, m, steps, segs, kind, variant):
+@pytest.mark.parametrize("Bd,kb,m,steps,segs,kind", SEGMENTED)
+def test_segmented(Bd, kb, m, steps, segs, kind):
     """A tensor list cut per tensor (each tensor's last block ragged) against the
     oracle's per-tensor cut."""
-    run_parity(sum(segs), Bd, kb, m, steps, kind=kind, segments=segs, variant=variant)
+    run_parity(sum(segs), Bd, kb, m, steps, kind=kind, segments=segs)
 
 
 def test_segmented_step():

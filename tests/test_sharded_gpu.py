@@ -1,10 +1,14 @@
-"""The sharded step on one GPU: two shard handles of one vector, run one after
-the other with the 8-byte (-delta, Delta) exchange done as a device-side MAX
-(what the all-reduce of a 2-rank run computes), must reproduce the unsharded
-step bit for bit: codes, window, scalars and parameters. No kernel waits on
-another; each launch completes on its own."""
+"""The sharded step on one GPU: shard handles of one vector, run one after the
+other with the 8-byte (-delta, Delta) exchange done as a device-side MAX (what
+the all-reduce of a multi-rank run computes), against the oracle run on the
+whole vector, every step: the shards' codes, window rows and scalars bit for
+bit, their parameters within 1e-5; and bit for bit against the unsharded
+step. No kernel waits on another; each launch completes on its own."""
+import numpy as np
 import pytest
 
+import oracle
+import state_view
 from conftest import cuda_available
 
 pytestmark = [pytest.mark.gpu,
@@ -22,6 +26,8 @@ def test_shards_reproduce_whole_vector(world):
     shards = [MicroAdam(d, block_size=Bd, k_per_block=kb, window=m,
                         shard=sharding.shard_blocks(d, Bd, r, world)) for r in range(world)]
     p0 = workloads.make_params(d).cuda()
+    ost = oracle.new_state(d, Bd, kb, m)
+    p_ref = p0.cpu().numpy().copy()
     p_whole = p0.clone()
     p_sh = [p0[s.offset: s.offset + s.d].clone() for s in shards]
     st_whole = whole.new_state()
@@ -40,8 +46,29 @@ def test_shards_reproduce_whole_vector(world):
             st[o:o + 8].view(torch.int32).copy_(pair)
         for s, p, gs, st in zip(shards, p_sh, g_sh, st_sh):
             s.apply(p, gs, st, t=t, **hyper)
+        oracle.step(ost, p_ref, workloads.bf16_bits(g), t=t, **hyper)
+        torch.cuda.synchronize()
+        # the shards, reassembled in the whole vector's layout, against the oracle
+        lw = whole.layout
+        sb = st_sh[0][:lw.codes].cpu().numpy().copy()
+        codes = torch.cat([st[s.layout.codes: s.layout.codes + s.d // 2 + (s.d % 2)]
+                           for s, st in zip(shards, st_sh)]).cpu().numpy()
+        win = torch.cat([st[s.layout.window: s.layout.bytes]
+                         for s, st in zip(shards, st_sh)]).cpu().numpy()
+        assert np.array_equal(codes, ost.codes), t
+        lo, hi = state_view.header_scalars(sb, t + 1)
+        assert np.float32(lo) == ost.scal[0] and np.float32(hi) == ost.scal[1], t
+        kp = lw.row_stride
+        wv = win.view(np.uint32).reshape(lw.blocks, m, kp)[:, :, :kb].transpose(1, 0, 2)
+        for s_ in range(max(1, t - m + 1), t + 1):
+            r = s_ % m
+            assert np.array_equal((wv[r] & 0xFFFF).astype(np.uint16).view(np.int16),
+                                  ost.G_idx[r]), (t, s_)
+            assert np.array_equal((wv[r] >> 16).astype(np.uint16), ost.G_val[r]), (t, s_)
+        p = torch.cat(p_sh).cpu().numpy().astype(np.float64)
+        tol = 1e-5 * np.maximum(np.abs(p_ref.astype(np.float64)), hyper["lr"])
+        assert np.all(np.abs(p - p_ref) <= tol), t
     torch.cuda.synchronize()
-    lw = whole.layout
     codes = torch.cat([st[s.layout.codes: s.layout.codes + s.d // 2 + (s.d % 2)]
                        for s, st in zip(shards, st_sh)])
     assert torch.equal(codes, st_whole[lw.codes: lw.codes + (d + 1) // 2])
