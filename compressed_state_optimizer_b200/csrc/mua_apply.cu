@@ -24,7 +24,8 @@ namespace {
 template <int T, bool VEC, bool FULL>
 __device__ __forceinline__ void codec_pass(const StepArgs& A, int64_t start, int base, int L,
                                            const uint32_t* sel, const char* lvb, float dn,
-                                           float inv16, const uint4 (&gv)[kChunks],
+                                           float inv16,
+                                           const uint4 (&gv)[kChunks],
                                            const uint32_t (&cv)[kChunks]) {
   const int tid = threadIdx.x;
   const Geometry& G = A.g;
@@ -42,14 +43,13 @@ __device__ __forceinline__ void codec_pass(const StepArgs& A, int64_t start, int
       const uint4 x = philox4x32_10((uint32_t)grp, (uint32_t)(grp >> 32), A.t_lo, A.t_hi, A.keys);
       uint64_t a2[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {  // elements 2i, 2i + 1: gradient word i
+      for (int i = 0; i < 4; ++i) {  // elements 2i, 2i + 1: gradient word i, code byte i
         const uint32_t w = chunk_word(gv[c], i);
-        const int e = 2 * i;
-        const uint32_t off0 = (e == 0) ? ((cv[c] << 2) & 0x3Cu) : ((cv[c] >> (4 * e - 2)) & 0x3Cu);
-        const uint32_t off1 = (cv[c] >> (4 * e + 2)) & 0x3Cu;
+        const uint32_t b = (cv[c] >> (8 * i)) & 0xFFu;
         const uint64_t g2 = ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint32_t)(w << 16);
-        const uint64_t l2 = f2_pack(*reinterpret_cast<const float*>(lvb + off0),
-                                    *reinterpret_cast<const float*>(lvb + off1));
+        const uint64_t l2 =
+            ((uint64_t)__float_as_uint(*reinterpret_cast<const float*>(lvb + 4 * (b >> 4))) << 32) |
+            __float_as_uint(*reinterpret_cast<const float*>(lvb + 4 * (b & 15u)));
         a2[i] = f2_add_rn(g2, l2);
       }
       pack = quantize8(a2, selbits, x, f2_pack(dn, dn), f2_pack(inv16, inv16));
@@ -105,6 +105,9 @@ __global__ void __launch_bounds__(T, (T == 256 ? MUA_APPLY_CTAS_256 : (T <= 512 
   // Every pass of a whole block lies inside it (B_d a multiple of the pass).
   const bool full = VEC && (L % kPass) == 0;
 
+  // The block's window rows start copying into shared memory now; they land
+  // while the codec runs (block_update waits for them).
+  update_prefetch_rows<T>(A, j, dyn);
   load_weights(A, s_w1, s_w2);
 
   uint32_t* sel = reinterpret_cast<uint32_t*>(dyn);  // [Wn] bits of the new row
@@ -118,7 +121,8 @@ __global__ void __launch_bounds__(T, (T == 256 ? MUA_APPLY_CTAS_256 : (T <= 512 
 
   const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
   const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
-  fill_levels(s_lv, delta, __fdiv_rn(__fsub_rn(Delta, delta), 15.0f));
+  const float unit = __fdiv_rn(__fsub_rn(Delta, delta), 15.0f);
+  fill_levels(s_lv, delta, unit);
   for (int w = tid; w < Wn; w += T) sel[w] = 0u;
   __syncthreads();
   {

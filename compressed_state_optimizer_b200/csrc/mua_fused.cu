@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   int64_t start;
   int L;
   block_span(A, j, start, L);
-  const int k = (int)(((int64_t)L * G.kb + G.Bd - 1) / G.Bd);
+  const int k = block_k(G, L);
   uint32_t* const status = &A.hdr[kHdrStatus];
 
   load_weights(A, S.w1, S.w2);
@@ -213,6 +213,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     __syncthreads();  // S.scan is reused by the next chunk's scan
   }
   for (int sl = k + tid; sl < G.kp; sl += T) row[sl] = kEmptySlot;
+  __syncthreads();  // the histogram is done with; the new row is written
+  update_prefetch_rows<T>(A, j, dyn);  // the window rows land during the barrier
 
   // (3) block min/max and the non-finite check, one atomic pair per CTA.
 #pragma unroll

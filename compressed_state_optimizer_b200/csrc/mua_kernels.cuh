@@ -85,6 +85,13 @@ struct StepArgs {
 // Start (element offset within the handle) and length of block j. Kernels
 // that call this take their StepArgs as a __grid_constant__ argument, so the
 // indexed reads stay in the parameter bank.
+// Entries a block of L parameters keeps: ceil(L k_b / B_d), k_b for a whole
+// block (L k_b < 2^30 since B_d <= 32766, so 32-bit arithmetic is exact).
+__device__ __forceinline__ int block_k(const Geometry& G, int L) {
+  if (L == G.Bd) return G.kb;
+  return (int)(((uint32_t)L * (uint32_t)G.kb + (uint32_t)G.Bd - 1u) / (uint32_t)G.Bd);
+}
+
 __device__ __forceinline__ void block_span(const StepArgs& A, int j, int64_t& start, int& L) {
   const Geometry& G = A.g;
   if (A.n_seg == 0) {
@@ -144,6 +151,20 @@ __device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
   uint32_t v;
   asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
+}
+__device__ __forceinline__ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// L2 prefetch hint for n bytes at p, issued only where `on` holds: no
+// destination, no completion to wait for. p and n must be multiples of 16
+// and the range must lie inside one allocation.
+__device__ __forceinline__ void prefetch_l2_if(bool on, const void* p, uint32_t n) {
+  asm volatile(
+      "{\n"
+      " .reg .pred q;\n"
+      " setp.ne.b32 q, %2, 0;\n"
+      " @q cp.async.bulk.prefetch.L2.global [%0], %1;\n"
+      "}\n" ::"l"(p), "r"(n), "r"((uint32_t)on)
+      : "memory");
 }
 // A 4-byte load of data this kernel also writes (the apply kernel's codes,
 // which it overwrites in place): not through the read-only path.
@@ -324,7 +345,9 @@ __device__ __forceinline__ V block_scan_1bar(V x, V* scratch, V& total) {
 
 // ---------------------------------------------------------------- Philox
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) with precomputed round
-// keys. Counter (c0, c1, c2, c3); returns the four output words.
+// keys (keys[r] = the key bumped r times by the Weyl constants; the kernel
+// argument block holds them, so each round's key is a constant-bank operand).
+// Counter (c0, c1, c2, c3); returns the four output words.
 __device__ __forceinline__ uint4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2,
                                                uint32_t c3, const uint32_t (&keys)[10][2]) {
   constexpr uint32_t M0 = 0xD2511F53u;
@@ -357,6 +380,16 @@ __device__ __forceinline__ float rcp_approx(float x) {
 }
 
 // ---------------------------------------------------------------- AdamStats + update
+
+// Asynchronous 16-byte global -> shared copies (cp.async, completed by the
+// hardware; waiting on them is a wait_group, not a spin).
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Shared-memory layout of block_update (dynamic):
 //   mask  u32[WnP]    bitmask of the window's index union (WnP = words padded to 4)
 //   wpre  u16[WnP8]   exclusive popcount prefix of mask (union rank of each word)
@@ -372,6 +405,32 @@ __host__ __device__ inline uint32_t update_smem_bytes(int threads, int Bd, int k
   const int E = m * kp;
   const int Ucap = Bd < E ? Bd : E;
   return (uint32_t)(4 * WnP + 2 * ((WnP + 7) & ~7) + 4 * E + 10 * Ucap + 4 * (threads / 32));
+}
+
+// Byte offset of W (the staged rows) in block_update's shared memory.
+__host__ __device__ inline uint32_t update_rows_offset(int Bd) {
+  const int WnP = mask_words_padded(Bd);
+  return (uint32_t)(4 * WnP + 2 * ((WnP + 7) & ~7));
+}
+
+// Starts copying block j's window rows of steps t, t-1, ..., t-rows+1 (age
+// 0 first) into W, 16 bytes at a time: rows are kp = 4q entries long and
+// start on 16-byte boundaries, so a copy never straddles two rows. The copies
+// complete in the background; block_update waits for them. W must not be
+// touched until then.
+template <int T>
+__device__ __forceinline__ void update_prefetch_rows(const StepArgs& A, int j, uint8_t* smem) {
+  const Geometry& G = A.g;
+  const uint32_t W = smem_addr(smem + update_rows_offset(G.Bd));
+  const uint32_t* wblk = A.window + (int64_t)j * G.m * G.kp;
+  const int staged4 = (A.rows * G.kp) >> 2;
+  for (int v = threadIdx.x; v < staged4; v += T) {
+    const int e = 4 * v;
+    const int age = (int)__umulhi((uint32_t)e, A.kp_recip);
+    int phys = A.row - age;
+    if (phys < 0) phys += G.m;
+    cp_async16(W + 16u * (uint32_t)v, wblk + phys * G.kp + (e - age * G.kp));
+  }
 }
 
 // Stage (6) for block j [MicroAdam ¶1]: m_hat = AdamStats(beta1, G) and
@@ -403,35 +462,17 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   uint32_t* scan = reinterpret_cast<uint32_t*>(uidx + Ucap);
 
   for (int w = tid; w < Wn; w += T) mask[w] = 0u;
-  __syncthreads();
+  cp_async_wait_all();  // this thread's copies of the rows (update_prefetch_rows)
+  __syncthreads();      // everyone's
 
-  // Rows of steps t, t-1, ..., t-rows+1 (age 0 = this step's row), staged 4
-  // entries (16 bytes) per load: rows are kp = 4q entries long and start on
-  // 16-byte boundaries, so a load never straddles two rows.
-  const uint32_t* wblk = A.window + (int64_t)j * G.m * G.kp;
+  // The union of the staged rows' indices.
   const int staged4 = (A.rows * G.kp) >> 2;
-  for (int v0 = tid; v0 < staged4; v0 += 2 * T) {
-    uint4 v[2];
+  for (int v = tid; v < staged4; v += T) {
+    const uint4 x = reinterpret_cast<const uint4*>(W)[v];
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {  // loads first, then the bookkeeping
-      const int e = 4 * (v0 + b * T);
-      v[b] = make_uint4(kEmptySlot, kEmptySlot, kEmptySlot, kEmptySlot);
-      if (v0 + b * T < staged4) {
-        const int age = (int)__umulhi((uint32_t)e, A.kp_recip);
-        int phys = A.row - age;
-        if (phys < 0) phys += G.m;
-        v[b] = *reinterpret_cast<const uint4*>(wblk + phys * G.kp + (e - age * G.kp));
-      }
-    }
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      if (v0 + b * T >= staged4) continue;
-      reinterpret_cast<uint4*>(W)[v0 + b * T] = v[b];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t idx = chunk_word(v[b], q) & 0xFFFFu;
-        if (idx < (uint32_t)L) atomicOr(&mask[idx >> 5], 1u << (idx & 31));  // 0xFFFF: empty
-      }
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t idx = chunk_word(x, q) & 0xFFFFu;
+      if (idx < (uint32_t)L) atomicOr(&mask[idx >> 5], 1u << (idx & 31));  // 0xFFFF: empty
     }
   }
   __syncthreads();
@@ -475,6 +516,18 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
   }
   __syncthreads();
 
+  // The parameters of this thread's first kPre union slots are loaded now,
+  // so that their latency overlaps the sums.
+  constexpr int kPre = 6;
+  uint32_t pidx[kPre];
+  float pv0[kPre];
+#pragma unroll
+  for (int b = 0; b < kPre; ++b) {
+    const uint32_t r = (uint32_t)(b * T + tid);
+    pidx[b] = (r < U) ? (uint32_t)uidx[r] : kNil;
+    pv0[b] = (r < U) ? load_param_sparse<BF16>(A, start + pidx[b]) : 0.0f;
+  }
+
   // The sums, one row at a time from the oldest: z <- z + beta^age * V.
   for (int age = A.rows - 1; age >= 0; --age) {
     const float c1 = s_w1[age], c2 = s_w2[age];
@@ -492,37 +545,38 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
     __syncthreads();
   }
 
-  // Parameter update on the union, up to kBatch slots per thread per round
-  // with all parameter loads issued before any store. u = m_hat/(eps+sqrt(v_hat))
-  // uses the hardware square root and reciprocal approximations (a few ulp,
-  // far inside the fp32 update's error).
+  // Parameter update on the union: u = m_hat/(eps+sqrt(v_hat)) with the
+  // hardware square root and reciprocal approximations (a few ulp, far inside
+  // the fp32 update's error). First the preloaded slots, then the rest up to
+  // kBatch slots per thread per round, all loads before any store.
+  auto update_slot = [&](uint32_t r, uint32_t idx, float p) {
+    const float2 z = acc[r];
+    const float mh = __fmul_rn(A.f1, z.x);
+    const float vh = __fmul_rn(A.f2, z.y);
+    if (A.has_decay) p = __fmul_rn(p, A.decay);
+    const float u = __fmul_rn(mh, rcp_approx(__fadd_rn(A.eps, sqrt_approx(vh))));
+    store_param<BF16>(A, start + idx, __fsub_rn(p, __fmul_rn(A.lr, u)));
+    if (A.mhat) {
+      A.mhat[start + idx] = mh;
+      A.vhat[start + idx] = vh;
+    }
+  };
+#pragma unroll
+  for (int b = 0; b < kPre; ++b)
+    if (pidx[b] != kNil) update_slot((uint32_t)(b * T + tid), pidx[b], pv0[b]);
   constexpr int kBatch = 4;
-  for (uint32_t r0 = 0; r0 < U; r0 += kBatch * T) {
+  for (uint32_t r0 = kPre * T; r0 < U; r0 += kBatch * T) {
     uint32_t idx[kBatch];
-    float mh[kBatch], vh[kBatch], pv[kBatch];
+    float pv[kBatch];
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
       const uint32_t r = r0 + (uint32_t)(b * T + tid);
-      idx[b] = kNil;
-      mh[b] = vh[b] = pv[b] = 0.0f;
-      if (r >= U) continue;
-      idx[b] = uidx[r];
-      const float2 z = acc[r];
-      mh[b] = __fmul_rn(A.f1, z.x);
-      vh[b] = __fmul_rn(A.f2, z.y);
-      pv[b] = load_param_sparse<BF16>(A, start + idx[b]);
-      if (A.has_decay) pv[b] = __fmul_rn(pv[b], A.decay);
+      idx[b] = (r < U) ? (uint32_t)uidx[r] : kNil;
+      pv[b] = (r < U) ? load_param_sparse<BF16>(A, start + idx[b]) : 0.0f;
     }
 #pragma unroll
-    for (int b = 0; b < kBatch; ++b) {
-      if (idx[b] == kNil) continue;
-      const float u = __fmul_rn(mh[b], rcp_approx(__fadd_rn(A.eps, sqrt_approx(vh[b]))));
-      store_param<BF16>(A, start + idx[b], __fsub_rn(pv[b], __fmul_rn(A.lr, u)));
-      if (A.mhat) {
-        A.mhat[start + idx[b]] = mh[b];
-        A.vhat[start + idx[b]] = vh[b];
-      }
-    }
+    for (int b = 0; b < kBatch; ++b)
+      if (idx[b] != kNil) update_slot(r0 + (uint32_t)(b * T + tid), idx[b], pv[b]);
   }
 }
 

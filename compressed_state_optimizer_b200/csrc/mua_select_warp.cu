@@ -2,40 +2,47 @@
 // paragraph 1 of "MicroAdam (Sparse-Gradient Adaptive Optimization with
 // Quantized Error Feedback)"):
 //   a_t = g_t + Q^{-1}(e_t, delta_t, Delta_t)      (streamed, never stored)
-//   (I_t, V_t) = Top-k of |a_t| (ties to the lower index), written in
-//   ascending index order to row t mod m of the window G,
+//   (I_t, V_t) = Top-k of |a_t| (ties to the lower index), written to row
+//   t mod m of the window G,
 //   the residual's block min/max folded into the global (-delta_{t+1},
 //   Delta_{t+1}) pair with one pair of integer atomics per block.
+// The order of the k pairs inside a row is not part of the method (the
+// AdamStats sums run per index, row by row); the kernel's order is fixed by
+// the data alone (see the candidate path).
 //
 // The blocks are independent, so a warp (not a CTA) owns one: no block-wide
-// barrier, and memory latency hides behind the other warps' blocks.
+// barrier, and memory latency hides behind the other warps' blocks. A CTA is
+// one warp by default: its shared memory is released as soon as its block is
+// done, whatever the other blocks on the SM take.
 //
 // Exact Top-k:
-//  * candidate path (blocks of 1024 to 32 * MASKW entries, k <= L/8):
+//  * candidate path (blocks of 1024 to LMAX entries, k <= L/8):
 //    512 sample keys (64 chunks of 8 spread over the block), each lane's top
 //    two, a warp sort of those 64 values -> tau_lo. One streaming pass (lane l
 //    holds elements 256 s + 8 l .. + 7 of step s) tests each |a| against the
 //    lane's threshold and appends the candidates {bits of a, index} to the
-//    lane's own strided region with one predicated 8-byte store; nothing else
-//    happens per element. A lane whose region fills drops its smallest keys
-//    and raises its threshold above them (make_room). An exact warp radix
-//    select over the candidates (8-bit digits from the highest bit where
-//    tau_lo and the largest candidate differ) gives the k-th key; the result
-//    is exact iff every raised lane threshold is at most that key (else the
-//    block takes the fallback). The selected entries are marked in a bitmask
-//    of the block (ties at the threshold by a lowest-index merge of the
-//    lanes' regions), and a popcount prefix of the mask gives each its place
-//    in the row;
-//  * residual min/max without a per-element cost: every element that was not
-//    appended has |a| below T, the largest lane threshold. The candidates that
+//    lane's own strided region with one predicated 4-byte and one 2-byte
+//    store; nothing else happens per element. A lane whose region fills
+//    drops its smallest keys and raises its threshold above them
+//    (make_room). An exact warp radix select over the candidates (8-bit
+//    digits from the highest bit where tau_lo and the largest candidate
+//    differ) gives the k-th key; the result is exact iff every raised lane
+//    threshold is at most that key (else the block takes the fallback). Ties
+//    at the threshold go to the lowest indices by a merge of the lanes'
+//    regions (each ascends by index). The row holds lane 0's selected entries,
+//    then lane 1's, ..., each lane's in ascending index order;
+//  * residual min/max without a per-element cost: an element a lane did not
+//    append has |a| below that lane's final threshold. The candidates that
 //    were not selected (and the dropped ones) are folded into the block's min
-//    and max; if that max is >= T and that min <= -T, no other element can
-//    change them. Otherwise (rare: one-signed or degenerate blocks) one more
-//    pass over the block folds every unselected element;
+//    and max; if those reach past +-tau_lo, only the elements of lanes that
+//    raised their threshold beyond them can still change the result, and the
+//    warp folds just those lanes' elements; otherwise (rare: one-signed or
+//    degenerate blocks) one more pass over the block folds every unselected
+//    element;
 //  * fallback (blocks under 1024 entries, k > L/8, too few candidates after
 //    the retry, or a dropped key at or above the threshold): exact radix
 //    select on all keys by streaming passes over the block (it is in L2 by
-//    then), 8 bits per pass, then one placing pass.
+//    then), 8 bits per pass, then one placing pass (ascending index order).
 // HBM traffic per parameter: 2 B gradient + 0.5 B codes read; per selected
 // entry 4 B written.
 #include "mua_kernels.cuh"
@@ -43,13 +50,13 @@
 // Warps (= blocks in flight) per CTA and candidate slots per lane, for blocks
 // of up to 16384 entries (S) and up to 32768 entries (L).
 #ifndef MUA_SELECT_WARPS_S
-#define MUA_SELECT_WARPS_S 8
+#define MUA_SELECT_WARPS_S 1
 #endif
 #ifndef MUA_SELECT_CAP_S
 #define MUA_SELECT_CAP_S 32
 #endif
 #ifndef MUA_SELECT_MINB_S
-#define MUA_SELECT_MINB_S (MUA_SELECT_WARPS_S == 8 ? 2 : 4)  // CTAs per SM its smem allows
+#define MUA_SELECT_MINB_S (24 / MUA_SELECT_WARPS_S)  // up to 24 warps per SM (9 KB of shared memory each)
 #endif
 #ifndef MUA_SELECT_WARPS_L
 #define MUA_SELECT_WARPS_L 4
@@ -67,31 +74,34 @@ namespace {
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 constexpr uint32_t kKeyInf = 0x7F800000u;  // key of +-inf; every threshold stays <= it
 #ifndef MUA_SELECT_UNROLL
-#define MUA_SELECT_UNROLL 2
+#define MUA_SELECT_UNROLL 1
 #endif
 constexpr int kUnroll = MUA_SELECT_UNROLL;  // 256-element steps per load group
+// 256-element steps of a whole-step block that one lane asks L2 to fetch (a
+// bulk prefetch, no completion to wait for) before the threshold sample, so
+// the streaming pass finds them on chip. The default covers a 16384 block.
+#ifndef MUA_SELECT_PREFETCH_STEPS
+#define MUA_SELECT_PREFETCH_STEPS 64
+#endif
 
-// MASKW: words of the selection bitmask, which covers one block (512 for
-// blocks of up to 16384 entries, 1024 up to 32768). CAP: slots per lane.
-template <int MASKW, int CAP>
+// CAP: candidate slots per lane. A candidate takes 6 bytes (its a_t bits
+// and its block index in two arrays).
+template <int CAP>
 struct WarpSmem {
-  uint2 cand[CAP * 32];  // lane l's i-th candidate at [32 i + l]: {bits of a_t, index}
-  uint32_t mask[MASKW];  // selection bitmask; its first 256 words are the radix histogram
-  uint16_t wpre[MASKW];  // exclusive popcount prefix of the mask words
+  uint32_t ckey[CAP * 32];  // lane l's i-th candidate at [32 i + l]: bits of a_t
+  uint16_t cidx[CAP * 32];  // ... and its block-relative index
+  uint32_t hist[256];       // radix histogram
 };
 
-#ifndef MUA_SELECT_PAIR_TABLE
-#define MUA_SELECT_PAIR_TABLE 0
-#endif
-
-template <int MASKW, int CAP, int WARPS>
+template <int CAP, int WARPS>
 struct CtaSmem {
-  float levels[16];
-#if MUA_SELECT_PAIR_TABLE
-  float2 pairs[256];  // entry b: (level[b & 15], level[b >> 4]), one code byte
-#endif
-  WarpSmem<MASKW, CAP> w[WARPS];
+  WarpSmem<CAP> w[WARPS];
 };
+
+// The 16 dequantization levels of the step, one table per CTA. A namespace-
+// scope array has a fixed shared address: every lookup is one load at a
+// constant offset from the code's byte offset, in the out-of-line helpers too.
+__shared__ float s_levels[16];
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t x, int lane) {
 #pragma unroll
@@ -128,66 +138,68 @@ __device__ __forceinline__ void load_step(const uint16_t* __restrict__ grads,
   }
 }
 
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-#if MUA_SELECT_PAIR_TABLE
-__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
-  return v;
-}
-#endif
-
 // a_t of element e of a step: f32(g) + level[code]. The code word is read as
 // byte offsets into the level table (nibble * 4).
-__device__ __forceinline__ float dequant1(const uint4& gv, uint32_t cv, const float* lv, int e) {
-  const char* lb = reinterpret_cast<const char*>(lv);
+__device__ __forceinline__ float level_of(uint32_t cv, int e) {
   const uint32_t off = (e == 0) ? ((cv << 2) & 0x3Cu) : ((cv >> (4 * e - 2)) & 0x3Cu);
-  return __fadd_rn(__uint_as_float(grad_bits(gv, e)), *reinterpret_cast<const float*>(lb + off));
+  return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(s_levels) + off);
 }
-// The same with the level table given by its shared-window address (for code
-// outside the kernel body, where a generic pointer would not be known to
-// point into shared memory).
-__device__ __forceinline__ float dequant1_sa(const uint4& gv, uint32_t cv, uint32_t lv_sa, int e) {
-  const uint32_t off = (e == 0) ? ((cv << 2) & 0x3Cu) : ((cv >> (4 * e - 2)) & 0x3Cu);
-  return __fadd_rn(__uint_as_float(grad_bits(gv, e)), lds_f32(lv_sa + off));
+__device__ __forceinline__ float dequant1(const uint4& gv, uint32_t cv, int e) {
+  return __fadd_rn(__uint_as_float(grad_bits(gv, e)), level_of(cv, e));
+}
+// Elements 2i and 2i + 1 with one paired add (the same two roundings).
+__device__ __forceinline__ void dequant2(const uint4& gv, uint32_t cv, int i, float& a0, float& a1) {
+  const uint32_t w = chunk_word(gv, i);
+  const uint64_t g2 = ((uint64_t)(w & 0xFFFF0000u) << 32) | (uint32_t)(w << 16);
+  const uint64_t a2 = f2_add_rn(g2, f2_pack(level_of(cv, 2 * i), level_of(cv, 2 * i + 1)));
+  a0 = f2_lo(a2);
+  a1 = f2_hi(a2);
 }
 
 // Bits of a_t for the 8 elements of a step, +0 past L.
-__device__ __forceinline__ void dequant8(const uint4& gv, uint32_t cv, const float* lv, int e0,
-                                         int L, uint32_t (&ab)[kChunk]) {
+__device__ __forceinline__ void dequant8(const uint4& gv, uint32_t cv, int e0, int L,
+                                         uint32_t (&ab)[kChunk]) {
 #pragma unroll
-  for (int e = 0; e < kChunk; ++e)
-    ab[e] = (e0 + e < L) ? __float_as_uint(dequant1(gv, cv, lv, e)) : 0u;
+  for (int e = 0; e < kChunk; ++e) ab[e] = (e0 + e < L) ? __float_as_uint(dequant1(gv, cv, e)) : 0u;
 }
 
-// Shared-memory accesses of one candidate slot by its 32-bit shared-window
-// address. The candidate regions are touched through these two only, and a
-// lane only ever touches its own region, so the volatile asm statements (kept
-// in program order) are all the ordering they need.
-__device__ __forceinline__ void sts_u2(uint32_t addr, uint32_t x, uint32_t y) {
-  asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(x), "r"(y));
+// Shared-memory accesses of one candidate by the 32-bit shared-window
+// addresses of its key and index slots (the 16-bit index moves through a
+// 32-bit register, which PTX allows for narrow loads and stores) (the index slot sits at a fixed
+// distance, half the key's offset, in its own array). The candidate regions are
+// touched through these only, and a lane only ever touches its own region, so
+// the volatile asm statements (kept in program order) are all the ordering
+// they need. A candidate is read back as {key bits, index}, or as its key
+// (|a| bits) alone.
+__device__ __forceinline__ void sts_cand(uint32_t ka, uint32_t ia, uint32_t bits, uint32_t idx) {
+  asm volatile("st.shared.b32 [%0], %2;\n st.shared.b16 [%1], %3;"
+               ::"r"(ka), "r"(ia), "r"(bits), "r"(idx));
 }
-__device__ __forceinline__ uint2 lds_u2(uint32_t addr) {
-  uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-  return v;
+__device__ __forceinline__ uint32_t lds_key(uint32_t ka) {
+  uint32_t k;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(k) : "r"(ka));
+  return k & 0x7FFFFFFFu;
+}
+__device__ __forceinline__ uint2 lds_cand(uint32_t ka, uint32_t ia) {
+  uint32_t k, i;
+  asm volatile("ld.shared.b32 %0, [%2];\n ld.shared.u16 %1, [%3];"
+               : "=r"(k), "=r"(i) : "r"(ka), "r"(ia));
+  return make_uint2(k, i);
 }
 
-// Per-lane state of the candidate pass. The lane's region is slots
-// base + 256 i (8-byte slots, the 32 lanes interleaved).
+// Per-lane state of the candidate pass. The lane's region is key slots
+// base + 128 i and index slots ibase + 64 i (the 32 lanes interleaved).
 template <int CAP>
 struct Lane {
-  uint32_t slot;    // shared address of the next free slot
-  uint32_t base;    // shared address of the lane's first slot
+  uint32_t slot;    // shared address of the next free key slot
+  uint32_t islot;   // ... and of the next free index slot
+  uint32_t base;    // shared address of the lane's first key slot
+  uint32_t ibase;   // ... and of its first index slot
   uint32_t tau;     // candidate threshold key (>= the warp's tau_lo, <= kKeyInf)
   float tau_f;      // the same threshold as a float: |a| >= tau_f <=> key >= tau
   float rmin, rmax; // min / max of the entries make_room dropped
-  __device__ __forceinline__ int count() const { return (int)((slot - base) >> 8); }
-  __device__ __forceinline__ bool full() const { return slot > base + 256u * (CAP - kChunk); }
+  __device__ __forceinline__ int count() const { return (int)((slot - base) >> 7); }
+  __device__ __forceinline__ bool full() const { return slot > base + 128u * (CAP - kChunk); }
 };
 
 // Makes room in a lane's region for one more 8-element step: while it holds
@@ -200,66 +212,60 @@ __device__ __noinline__ Lane<CAP> make_room(Lane<CAP> st, uint32_t* status) {
   while (st.full()) {
     const int n = st.count();
     uint32_t m0 = kFull;
-    for (int i = 0; i < n; ++i) m0 = min(m0, lds_u2(st.base + 256u * i).x & 0x7FFFFFFFu);
-    uint32_t kept = st.base;
+    for (int i = 0; i < n; ++i)
+      m0 = min(m0, lds_cand(st.base + 128u * i, st.ibase + 64u * i).x & 0x7FFFFFFFu);
+    uint32_t kept = 0u;
     for (int i = 0; i < n; ++i) {
-      const uint2 e = lds_u2(st.base + 256u * i);
+      const uint2 e = lds_cand(st.base + 128u * i, st.ibase + 64u * i);
       if ((e.x & 0x7FFFFFFFu) == m0) {
         st.rmin = fminf(st.rmin, __uint_as_float(e.x));
         st.rmax = fmaxf(st.rmax, __uint_as_float(e.x));
       } else {
-        sts_u2(kept, e.x, e.y);
-        kept += 256u;
+        sts_cand(st.base + 128u * kept, st.ibase + 64u * kept, e.x, e.y);
+        ++kept;
       }
     }
     if (m0 >= kKeyInf) atomicOr(status, kStatusNonFinite);
-    st.slot = kept;
+    st.slot = st.base + 128u * kept;
+    st.islot = st.ibase + 64u * kept;
     st.tau = max(st.tau, min(m0 + 1u, kKeyInf));
     st.tau_f = __uint_as_float(st.tau);
   }
   return st;
 }
 
-// Appends {bits of a, idx} at `slot` and advances it by one slot (256 bytes)
-// iff |a| >= tau or a is NaN: one predicated compare, store and add, no branch.
-__device__ __forceinline__ void append_if(uint32_t& slot, float a, float tau, uint32_t idx) {
+// Appends {bits of a, idx} at the lane's next slots and advances them iff
+// |a| >= tau or a is NaN: one predicated compare, two stores and two adds, no
+// branch.
+__device__ __forceinline__ void append_if(uint32_t& slot, uint32_t& islot, float a, float tau,
+                                          uint32_t idx) {
   asm volatile(
       "{\n"
       " .reg .pred p;\n"
       " .reg .f32 t;\n"
-      " abs.f32 t, %1;\n"
-      " setp.geu.f32 p, t, %2;\n"
-      " @p st.shared.v2.b32 [%0], {%3, %4};\n"
-      " @p add.u32 %0, %0, 256;\n"
+      " abs.f32 t, %2;\n"
+      " setp.geu.f32 p, t, %3;\n"
+      " @p st.shared.b32 [%0], %4;\n"
+      " @p st.shared.b16 [%1], %5;\n"
+      " @p add.u32 %0, %0, 128;\n"
+      " @p add.u32 %1, %1, 64;\n"
       "}\n"
-      : "+r"(slot)
+      : "+r"(slot), "+r"(islot)
       : "f"(a), "f"(tau), "r"(__float_as_uint(a)), "r"(idx));
 }
 
 // The streaming test of one step: every |a| >= the lane's threshold (NaN
 // included) is appended. FULL: all 8 elements lie inside the block.
 template <int CAP, bool FULL>
-__device__ __forceinline__ void scan_step(const uint4& gv, uint32_t cv, uint32_t lv_sa, int e0,
-                                          int L, Lane<CAP>& st, uint32_t* status) {
+__device__ __forceinline__ void scan_step(const uint4& gv, uint32_t cv, int e0, int L,
+                                          Lane<CAP>& st, uint32_t* status) {
   if (st.full()) st = make_room(st, status);
   float a[kChunk];
-#if MUA_SELECT_PAIR_TABLE
-  // lv_sa is the pair table: one 8-byte load per code byte (two elements)
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t off = (i == 0) ? ((cv << 3) & 0x7F8u) : ((cv >> (8 * i - 3)) & 0x7F8u);
-    const float2 lev = lds_f2(lv_sa + off);
-    const uint32_t w = chunk_word(gv, i);
-    a[2 * i] = __fadd_rn(__uint_as_float(w << 16), lev.x);
-    a[2 * i + 1] = __fadd_rn(__uint_as_float(w & 0xFFFF0000u), lev.y);
-  }
-#else
-#pragma unroll
-  for (int e = 0; e < kChunk; ++e) a[e] = dequant1_sa(gv, cv, lv_sa, e);
-#endif
+  for (int i = 0; i < kChunk / 2; ++i) dequant2(gv, cv, i, a[2 * i], a[2 * i + 1]);
 #pragma unroll
   for (int e = 0; e < kChunk; ++e) {
-    if (FULL || e0 + e < L) append_if(st.slot, a[e], st.tau_f, (uint32_t)(e0 + e));
+    if (FULL || e0 + e < L) append_if(st.slot, st.islot, a[e], st.tau_f, (uint32_t)(e0 + e));
   }
 }
 
@@ -268,8 +274,8 @@ __device__ __forceinline__ void scan_step(const uint4& gv, uint32_t cv, uint32_t
 // step. Kept out of line: the retry calls it again.
 template <bool VEC, int CAP>
 __device__ __noinline__ Lane<CAP> stream_candidates(const StepArgs& A, int64_t start, int L,
-                                                    uint32_t lv_sa, uint32_t tau_lo,
-                                                    uint32_t base, int lane) {
+                                                    uint32_t tau_lo,
+                                                    uint32_t base, uint32_t ibase, int lane) {
   // The argument block is read once: after a call to make_room the compiler
   // would otherwise reload these from parameter space on every step.
   uint32_t* const status = &A.hdr[kHdrStatus];
@@ -277,6 +283,7 @@ __device__ __noinline__ Lane<CAP> stream_candidates(const StepArgs& A, int64_t s
   const uint8_t* const codes = A.codes;
   Lane<CAP> st;
   st.base = st.slot = base;
+  st.ibase = st.islot = ibase;
   st.tau = tau_lo;
   st.tau_f = __uint_as_float(tau_lo);
   st.rmin = st.rmax = 0.0f;
@@ -299,7 +306,7 @@ __device__ __noinline__ Lane<CAP> stream_candidates(const StepArgs& A, int64_t s
     auto run_full = [&](const uint4 (&g)[kUnroll], const uint32_t (&c)[kUnroll], int s0) {
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u)
-        scan_step<CAP, true>(g[u], c[u], lv_sa, ((s0 + u) << 8) + 8 * lane, L, st, status);
+        scan_step<CAP, true>(g[u], c[u], ((s0 + u) << 8) + 8 * lane, L, st, status);
     };
     load_full(ga, ca, 0);
     for (int s0 = 0; s0 < nfull; s0 += 2 * kUnroll) {
@@ -320,7 +327,7 @@ __device__ __noinline__ Lane<CAP> stream_candidates(const StepArgs& A, int64_t s
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u)
       if (s0 + u < nfull)
-        scan_step<CAP, true>(g[u], c[u], lv_sa, ((s0 + u) << 8) + 8 * lane, L, st, status);
+        scan_step<CAP, true>(g[u], c[u], ((s0 + u) << 8) + 8 * lane, L, st, status);
   };
   load_group(ga, ca, 0);
   for (int s0 = 0; s0 < nfull; s0 += 2 * kUnroll) {
@@ -334,7 +341,7 @@ __device__ __noinline__ Lane<CAP> stream_candidates(const StepArgs& A, int64_t s
     uint4 gv;
     uint32_t cv;
     load_step<VEC>(grads, codes, start, L, e0, gv, cv);
-    scan_step<CAP, false>(gv, cv, lv_sa, e0, L, st, status);
+    scan_step<CAP, false>(gv, cv, e0, L, st, status);
   }
   return st;
 }
@@ -427,7 +434,7 @@ __device__ __forceinline__ void warp_radix(int hi, uint32_t prefix, int k, uint3
 // lane r / 2, slot r % 2). Returns the keys at rank `r` and at rank 63.
 template <bool VEC>
 __device__ __forceinline__ void sample_threshold(const StepArgs& A, int64_t start, int L,
-                                                 const float* lv, int r, int lane,
+                                                 int r, int lane,
                                                  uint32_t& tau_first, uint32_t& tau_retry) {
   const int cstride = (L / 64) & ~7;
   uint32_t t1 = 0u, t2 = 0u;
@@ -438,7 +445,7 @@ __device__ __forceinline__ void sample_threshold(const StepArgs& A, int64_t star
     uint32_t cv;
     load_step<VEC>(A.grads, A.codes, start, L, e0, gv, cv);
     uint32_t ab[kChunk];
-    dequant8(gv, cv, lv, e0, L, ab);
+    dequant8(gv, cv, e0, L, ab);
 #pragma unroll
     for (int e = 0; e < kChunk; ++e) {
       const uint32_t key = ab[e] & 0x7FFFFFFFu;
@@ -473,50 +480,82 @@ __device__ __forceinline__ void sample_threshold(const StepArgs& A, int64_t star
   tau_retry = min(__shfl_sync(kFull, v1, 31), kKeyInf);  // the smallest of the 64
 }
 
-template <bool VEC, int MASKW, int CAP, int WARPS, int MINB>
+// Folds unselected elements into the lane's residual min/max: those of the
+// lanes in `open` (each lane's eight-element chunk of every 256-element step,
+// spread over the warp), or every element of the block when `open` is 0. An
+// element is selected iff its key is above thr, or equals it with an index
+// below its owner lane's `cut`.
+template <bool VEC>
+__device__ __noinline__ void fold_unselected(const StepArgs& A, int64_t start, int L,
+                                             uint32_t thr, uint32_t cut, uint32_t open,
+                                             int lane, float& rmin, float& rmax) {
+  const int nsteps = (L + 255) >> 8;
+  auto fold_step = [&](int e0, uint32_t c) {  // the unselected elements e0 .. e0 + 7
+    uint4 gv;
+    uint32_t cv;
+    load_step<VEC>(A.grads, A.codes, start, L, e0, gv, cv);
+    uint32_t ab[kChunk];
+    dequant8(gv, cv, e0, L, ab);
+#pragma unroll
+    for (int e = 0; e < kChunk; ++e) {
+      const uint32_t key = ab[e] & 0x7FFFFFFFu;
+      if (e0 + e >= L || key > thr || (key == thr && (uint32_t)(e0 + e) < c)) continue;
+      rmin = fminf(rmin, __uint_as_float(ab[e]));
+      rmax = fmaxf(rmax, __uint_as_float(ab[e]));
+    }
+  };
+  if (open == 0u) {
+    for (int s = 0; s < nsteps; ++s) fold_step((s << 8) + 8 * lane, cut);
+    return;
+  }
+  while (open) {
+    const int l = __ffs(open) - 1;
+    open &= open - 1;
+    const uint32_t cl = __shfl_sync(kFull, cut, l);
+    for (int s = lane; s < nsteps; s += 32) fold_step((s << 8) + 8 * l, cl);
+  }
+}
+
+template <bool VEC, int LMAX, int CAP, int WARPS, int MINB>
 __global__ void __launch_bounds__(WARPS * 32, MINB)
     mua_select_warp_kernel(const __grid_constant__ StepArgs A) {
   extern __shared__ __align__(16) uint8_t dyn[];
-  CtaSmem<MASKW, CAP, WARPS>& S = *reinterpret_cast<CtaSmem<MASKW, CAP, WARPS>*>(dyn);
+  CtaSmem<CAP, WARPS>& S = *reinterpret_cast<CtaSmem<CAP, WARPS>*>(dyn);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const Geometry& G = A.g;
   {
     const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
     const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
     const float unit = __fdiv_rn(__fsub_rn(Delta, delta), 15.0f);
-    fill_levels(S.levels, delta, unit);
-#if MUA_SELECT_PAIR_TABLE
-    for (int b = threadIdx.x; b < 256; b += WARPS * 32) {
-      const float c0 = __fsub_rn(__uint_as_float(0x4B000000u | (uint32_t)(b & 15)), 8388608.0f);
-      const float c1 = __fsub_rn(__uint_as_float(0x4B000000u | (uint32_t)(b >> 4)), 8388608.0f);
-      S.pairs[b] = make_float2(__fadd_rn(delta, __fmul_rn(c0, unit)),
-                               __fadd_rn(delta, __fmul_rn(c1, unit)));
-    }
-#endif
+    fill_levels(s_levels, delta, unit);
   }
-  __syncthreads();  // the only CTA barrier: the level tables
+  __syncthreads();  // the only CTA barrier: the level table
   const int j = blockIdx.x * WARPS + wid;
   if (j >= G.nb) return;
-  WarpSmem<MASKW, CAP>& W = S.w[wid];
-  const float* lv = S.levels;
+  WarpSmem<CAP>& W = S.w[wid];
   uint32_t* const status = &A.hdr[kHdrStatus];
   int64_t start;
   int L;
   block_span(A, j, start, L);
-  const int k = (int)(((int64_t)L * G.kb + G.Bd - 1) / G.Bd);
+  const int k = block_k(G, L);
   uint32_t* row = A.window + ((int64_t)j * G.m + A.row) * G.kp;
   const int nsteps = (L + 255) >> 8;
-  const int wn = (L + 31) >> 5;  // mask words of the block
 
   float rmin = 0.0f, rmax = 0.0f;  // residual; selected entries become +0
   bool done = false;
 
   // ---------------- candidate path
-  if (L >= 1024 && L <= 32 * MASKW && 8 * k <= L) {
+  if (L >= 1024 && L <= LMAX && 8 * k <= L) {
     // rank of tau_lo among the 64 sampled values: ~2.5 % of the block above it
-    const int r = min(63, (int)((1280 * (int64_t)k + L - 1) / L) - 1);
+    const int r = min(63, (int)((1280u * (uint32_t)k + (uint32_t)L - 1u) / (uint32_t)L) - 1);
+    if (VEC && (L & 255) == 0) {  // the streaming pass's data, on its way into L2
+      const int n = min(MUA_SELECT_PREFETCH_STEPS, L >> 8);
+      const bool pf = lane == 0 && aligned16(A.grads + start) && aligned16(A.codes + (start >> 1));
+      prefetch_l2_if(pf, A.grads + start, 512u * n);
+      prefetch_l2_if(pf, A.codes + (start >> 1), 128u * n);
+    }
     uint32_t tau_first, tau_retry;
-    sample_threshold<VEC>(A, start, L, lv, r, lane, tau_first, tau_retry);
+    sample_threshold<VEC>(A, start, L, r, lane, tau_first, tau_retry);
 
     // One streaming pass per attempt (a second, with a lower tau_lo, only when
     // the first finds fewer than k candidates). An all-zero sample goes
@@ -524,117 +563,102 @@ __global__ void __launch_bounds__(WARPS * 32, MINB)
     for (int attempt = 0; attempt < 2 && !done && tau_first != 0u; ++attempt) {
       const uint32_t tau_lo = attempt == 0 ? tau_first : tau_retry;
       if (attempt == 1 && tau_retry >= tau_first) break;
-#if MUA_SELECT_PAIR_TABLE
-      const uint32_t stream_lv = smem_addr(S.pairs);
-#else
-      const uint32_t stream_lv = smem_addr(S.levels);
-#endif
-      const Lane<CAP> st = stream_candidates<VEC, CAP>(A, start, L, stream_lv, tau_lo,
-                                                       smem_addr(&W.cand[lane]), lane);
+      const Lane<CAP> st = stream_candidates<VEC, CAP>(
+          A, start, L, tau_lo, smem_addr(&W.ckey[lane]), smem_addr(&W.cidx[lane]), lane);
       const int mine = st.count();
       const uint32_t n = __reduce_add_sync(kFull, (uint32_t)mine);
       const uint32_t drop_bound = __reduce_max_sync(kFull, st.tau > tau_lo ? st.tau : 0u);
       const uint32_t T = __reduce_max_sync(kFull, st.tau);  // every non-candidate key < T
       if (n < (uint32_t)k) continue;  // too few: retry lower, else the fallback
-      const uint32_t cand = st.base;  // the lane's i-th candidate at cand + 256 i
+      // the lane's i-th candidate: key slot cand + 128 i, index slot icand + 64 i
+      const uint32_t cand = st.base, icand = st.ibase;
+      auto entry = [&](int i) { return lds_cand(cand + 128u * i, icand + 64u * i); };
+      auto key_of = [&](int i) { return lds_key(cand + 128u * i); };
       uint32_t kmax = 0u;
-      for (int i = 0; i < mine; ++i) kmax = max(kmax, lds_u2(cand + 256u * i).x & 0x7FFFFFFFu);
+#pragma unroll 4
+      for (int i = 0; i < mine; ++i) kmax = max(kmax, key_of(i));
       kmax = __reduce_max_sync(kFull, kmax);
       int mode = 1, need = k;
       uint32_t thr = tau_lo;
       const uint32_t diff = kmax ^ tau_lo;
       if (diff != 0u) {
-        warp_radix(31 - __clz(diff), tau_lo, k, W.mask, lane,
+        warp_radix(31 - __clz(diff), tau_lo, k, W.hist, lane,
                    [&](auto&& f) {
-                     for (int i = 0; i < mine; ++i) f(lds_u2(cand + 256u * i).x & 0x7FFFFFFFu);
+#pragma unroll 4
+                     for (int i = 0; i < mine; ++i) f(key_of(i));
                    },
                    mode, thr, need);
       }
       // Exact only if every dropped key (< its lane's tau <= drop_bound) is below thr.
       if (drop_bound > thr) break;
       if (lane == 0 && kmax >= kKeyInf) atomicOr(status, kStatusNonFinite);
-      // Selection bitmask: keys above the threshold (at or above it in mode 0) ...
-      for (int w = lane; w < wn; w += 32) W.mask[w] = 0u;
-      __syncwarp();
-      for (int i = 0; i < mine; ++i) {
-        const uint2 e = lds_u2(cand + 256u * i);
-        const uint32_t key = e.x & 0x7FFFFFFFu;
-        if (mode == 0 ? key >= thr : key > thr) atomicOr(&W.mask[e.y >> 5], 1u << (e.y & 31));
-      }
-      // ... and, in mode 1, the `need` lowest indices among keys equal to it,
-      // one per round: the lowest unmarked tied index over all lanes.
+      // The selection: keys above thr, and keys equal to it (all of them in
+      // mode 0; in mode 1 the `need` lowest indices over the warp). A lane's
+      // entries ascend by index, so the ties a lane gives are a prefix of its
+      // ties: those below `cut`, its first tie left out (0x10000: none).
+      uint32_t cut = 0x10000u, won = 0u;
       if (mode == 1) {
-        for (int q = 0; q < need; ++q) {
-          __syncwarp();
-          uint32_t head = 0xFFFFu;
-          for (int i = 0; i < mine; ++i) {
-            const uint2 e = lds_u2(cand + 256u * i);
-            if ((e.x & 0x7FFFFFFFu) != thr) continue;
-            if (e.y < head && !((W.mask[e.y >> 5] >> (e.y & 31)) & 1u)) head = e.y;
+        int cur = 0;
+        auto next_tie = [&]() -> uint32_t {
+          for (; cur < mine; ++cur) {
+            const uint2 e = entry(cur);
+            if ((e.x & 0x7FFFFFFFu) == thr) return e.y;
           }
-          const uint32_t low = __reduce_min_sync(kFull, head);
-          if (head == low && head != 0xFFFFu) atomicOr(&W.mask[head >> 5], 1u << (head & 31));
-        }
-      }
-      __syncwarp();
-      // u16 exclusive popcount prefix of the mask words (lane l: words
-      // MASKW/32 l ..)
-      {
-        constexpr int kWpl = MASKW / 32;
-        const int w0 = kWpl * lane;
-        uint32_t c = 0u;
-#pragma unroll
-        for (int w = 0; w < kWpl; ++w) c += (w0 + w < wn) ? (uint32_t)__popc(W.mask[w0 + w]) : 0u;
-        uint32_t run = warp_incl_scan(c, lane) - c;
-#pragma unroll
-        for (int w = 0; w < kWpl; ++w) {
-          if (w0 + w < wn) {
-            W.wpre[w0 + w] = (uint16_t)run;
-            run += (uint32_t)__popc(W.mask[w0 + w]);
+          return 0x10000u;
+        };
+        uint32_t head = next_tie();
+        for (int q = 0; q < need; ++q) {  // one tie per round: the lowest head
+          if (head == __reduce_min_sync(kFull, head)) {
+            ++won;
+            ++cur;
+            head = next_tie();
           }
         }
+        cut = head;
       }
-      __syncwarp();
+      // The row, lane by lane (each lane's entries in ascending index order):
+      // a lane's first place is the count of entries the lanes below it give.
+      uint32_t nsel = won;
+#pragma unroll 4
+      for (int i = 0; i < mine; ++i) {
+        const uint32_t key = key_of(i);
+        nsel += (key > thr || (mode == 0 && key == thr)) ? 1u : 0u;
+      }
+      uint32_t pos = warp_incl_scan(nsel, lane) - nsel;
       // Place the selected entries; the others join the residual's min/max.
       rmin = st.rmin;
       rmax = st.rmax;
       for (int i = 0; i < mine; ++i) {
-        const uint2 e = lds_u2(cand + 256u * i);
-        const uint32_t word = W.mask[e.y >> 5];
-        if ((word >> (e.y & 31)) & 1u) {
-          const uint32_t pos = W.wpre[e.y >> 5] + (uint32_t)__popc(word & ((1u << (e.y & 31)) - 1u));
+        const uint2 e = entry(i);
+        const uint32_t key = e.x & 0x7FFFFFFFu;
+        if (key > thr || (key == thr && e.y < cut)) {
           put_row(row, pos, k, e.y, e.x);
+          ++pos;
         } else {
           rmin = fminf(rmin, __uint_as_float(e.x));
           rmax = fmaxf(rmax, __uint_as_float(e.x));
         }
       }
-      // Elements never appended have |a| < T: they can only move the min or
-      // the max if the folded values do not reach past +-T.
-      const float Tf = __uint_as_float(T);
+      // Elements a lane never appended have |a| below that lane's final
+      // threshold: tau_lo for lanes that never raised it. If the folded values
+      // reach past +-tau_lo, only raised lanes whose threshold is beyond them
+      // can still move the min or the max: their own elements are folded (two
+      // steps per warp lane). Otherwise (rare: one-signed or degenerate blocks)
+      // every unselected element of the block is.
       float bmin = rmin, bmax = rmax;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         bmin = fminf(bmin, __shfl_xor_sync(kFull, bmin, o));
         bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
       }
-      if (!(bmax >= Tf && bmin <= -Tf)) {
-        // One more pass: every unselected element of the block.
-        for (int s = 0; s < nsteps; ++s) {
-          const int e0 = (s << 8) + 8 * lane;
-          uint4 gv;
-          uint32_t cv;
-          load_step<VEC>(A.grads, A.codes, start, L, e0, gv, cv);
-          uint32_t ab[kChunk];
-          dequant8(gv, cv, lv, e0, L, ab);
-          const uint32_t sel = (e0 < L) ? (W.mask[e0 >> 5] >> (e0 & 31)) : 0xFFu;
-#pragma unroll
-          for (int e = 0; e < kChunk; ++e) {
-            if (e0 + e >= L || ((sel >> e) & 1u)) continue;
-            rmin = fminf(rmin, __uint_as_float(ab[e]));
-            rmax = fmaxf(rmax, __uint_as_float(ab[e]));
-          }
-        }
+      const float lo_f = __uint_as_float(tau_lo);
+      if (bmax >= lo_f && bmin <= -lo_f) {
+        const float mine_f = __uint_as_float(st.tau);
+        const uint32_t open =
+            __ballot_sync(kFull, st.tau > tau_lo && !(bmax >= mine_f && bmin <= -mine_f));
+        if (open) fold_unselected<VEC>(A, start, L, thr, cut, open, lane, rmin, rmax);
+      } else {
+        fold_unselected<VEC>(A, start, L, thr, cut, 0u, lane, rmin, rmax);
       }
       done = true;
     }
@@ -652,12 +676,12 @@ __global__ void __launch_bounds__(WARPS * 32, MINB)
         uint32_t cv;
         load_step<VEC>(A.grads, A.codes, start, L, e0, gv, cv);
         uint32_t ab[kChunk];
-        dequant8(gv, cv, lv, e0, L, ab);
+        dequant8(gv, cv, e0, L, ab);
 #pragma unroll
         for (int e = 0; e < kChunk; ++e) f(ab[e] & 0x7FFFFFFFu);
       }
     };
-    warp_radix(30, 0u, k, W.mask, lane, stream_keys, mode, thr, need);
+    warp_radix(30, 0u, k, W.hist, lane, stream_keys, mode, thr, need);
     uint32_t run_g = 0u, run_e = 0u;  // warp-uniform running counts
     uint32_t kmax = 0u;
     for (int s = 0; s < nsteps; ++s) {
@@ -666,7 +690,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB)
       uint32_t cv;
       load_step<VEC>(A.grads, A.codes, start, L, e0, gv, cv);
       uint32_t ab[kChunk];
-      dequant8(gv, cv, lv, e0, L, ab);
+      dequant8(gv, cv, e0, L, ab);
       uint32_t cg = 0u, ce = 0u;
 #pragma unroll
       for (int e = 0; e < kChunk; ++e) {
@@ -722,10 +746,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB)
   }
 }
 
-template <bool VEC, int MASKW, int CAP, int WARPS, int MINB>
+template <bool VEC, int LMAX, int CAP, int WARPS, int MINB>
 cudaError_t launch_shape(const StepArgs& args, cudaStream_t stream) {
-  auto kern = mua_select_warp_kernel<VEC, MASKW, CAP, WARPS, MINB>;
-  const uint32_t smem = (uint32_t)sizeof(CtaSmem<MASKW, CAP, WARPS>);
+  auto kern = mua_select_warp_kernel<VEC, LMAX, CAP, WARPS, MINB>;
+  const uint32_t smem = (uint32_t)sizeof(CtaSmem<CAP, WARPS>);
   static uint32_t opted[kMaxDevices] = {};
   const cudaError_t e = opt_in_smem(kern, smem, opted);
   if (e != cudaSuccess) return e;
@@ -738,19 +762,19 @@ cudaError_t launch_shape(const StepArgs& args, cudaStream_t stream) {
 
 uint32_t select_warp_smem_bytes(int Bd) {
   return Bd <= 16384
-             ? (uint32_t)sizeof(CtaSmem<512, MUA_SELECT_CAP_S, MUA_SELECT_WARPS_S>)
-             : (uint32_t)sizeof(CtaSmem<1024, MUA_SELECT_CAP_L, MUA_SELECT_WARPS_L>);
+             ? (uint32_t)sizeof(CtaSmem<MUA_SELECT_CAP_S, MUA_SELECT_WARPS_S>)
+             : (uint32_t)sizeof(CtaSmem<MUA_SELECT_CAP_L, MUA_SELECT_WARPS_L>);
 }
 
 cudaError_t launch_select_warp(const StepArgs& args, bool vec, cudaStream_t stream) {
   if (args.g.Bd > 16384)
-    return vec ? launch_shape<true, 1024, MUA_SELECT_CAP_L, MUA_SELECT_WARPS_L, MUA_SELECT_MINB_L>(
+    return vec ? launch_shape<true, 32768, MUA_SELECT_CAP_L, MUA_SELECT_WARPS_L, MUA_SELECT_MINB_L>(
                      args, stream)
-               : launch_shape<false, 1024, MUA_SELECT_CAP_L, MUA_SELECT_WARPS_L, MUA_SELECT_MINB_L>(
+               : launch_shape<false, 32768, MUA_SELECT_CAP_L, MUA_SELECT_WARPS_L, MUA_SELECT_MINB_L>(
                      args, stream);
-  return vec ? launch_shape<true, 512, MUA_SELECT_CAP_S, MUA_SELECT_WARPS_S, MUA_SELECT_MINB_S>(
+  return vec ? launch_shape<true, 16384, MUA_SELECT_CAP_S, MUA_SELECT_WARPS_S, MUA_SELECT_MINB_S>(
                    args, stream)
-             : launch_shape<false, 512, MUA_SELECT_CAP_S, MUA_SELECT_WARPS_S, MUA_SELECT_MINB_S>(
+             : launch_shape<false, 16384, MUA_SELECT_CAP_S, MUA_SELECT_WARPS_S, MUA_SELECT_MINB_S>(
                    args, stream);
 }
 

@@ -5,8 +5,9 @@ oracle can compute one block at a time.
 Blocks depend on each other only through delta_t / Delta_t. Before each
 step, a sample of blocks' state is read back from the device (codes, all
 window rows, parameters) with the global (delta_t, Delta_t); then:
-  * each sampled block's new window row and updated parameters equal the
-    oracle run on that block alone from that state (bit for bit / 1e-5);
+  * each sampled block's new window row (as a set of pairs) and updated
+    parameters equal the oracle run on that block alone from that state (bit
+    for bit / 1e-5);
   * delta_{t+1}, Delta_{t+1}: the min and max of the residual over the whole
     vector, computed independently with torch from the gradients, a device
     copy of the previous codes and the (row-verified) selection;
@@ -100,10 +101,9 @@ def check_steps_sampled(w, steps, n_random=27, need_bytes=0):
             p = b["p"].copy()
             oracle.step(ost, p, g, t=t, **hyper)
             gw = win[(j * m + row) * kp: (j * m + row) * kp + kb].cpu().numpy().view(np.uint32)
-            assert np.array_equal((gw & 0xFFFF).astype(np.uint16).view(np.int16),
-                                  ost.G_idx[row, 0]), f"t={t} block {j} indices"
-            assert np.array_equal((gw >> 16).astype(np.uint16), ost.G_val[row, 0]), \
-                f"t={t} block {j} values"
+            gi, gv = state_view.canonical_words(gw)
+            assert np.array_equal(gi, ost.G_idx[row, 0]), f"t={t} block {j} indices"
+            assert np.array_equal(gv, ost.G_val[row, 0]), f"t={t} block {j} values"
             pg = params[lo:lo + L].cpu().numpy().astype(np.float64)
             tol = 1e-5 * np.maximum(np.abs(p.astype(np.float64)), w.lr)
             assert np.all(np.abs(pg - p) <= tol), f"t={t} block {j} parameters"

@@ -1,9 +1,10 @@
 """GPU parity: the CUDA path (through the C ABI) against the CPU oracle, step by
 step, on the same seeded inputs.
 
-Bit-exact: the window rows (int16 I, bf16 V), the 4-bit codes, delta/Delta
-and the status word. Within 1e-5: the parameters (relative, with an absolute
-floor of 1e-5 * lr, the scale of one update), v_hat (relative) and m_hat
+Bit-exact: the window rows (int16 I, bf16 V; each row as a set of pairs, put
+in ascending index order), the 4-bit codes, delta/Delta and the status word.
+Within 1e-5: the parameters (relative, with an absolute floor of 1e-5 * lr,
+the scale of one update), v_hat (relative) and m_hat
 (relative to the cancellation-free magnitude (1-b1)/(1-b1^t) sum b1^r |V|,
 since m_hat sums terms of both signs).
 """
@@ -35,7 +36,7 @@ def compare_state(mo, state, ost, t, d, m, kb, what=""):
     lo, hi = state_view.header_scalars(sb, t + 1)
     assert np.float32(lo).view(np.uint32) == ost.scal[0:1].view(np.uint32)[0], (what, t, lo, ost.scal)
     assert np.float32(hi).view(np.uint32) == ost.scal[1:2].view(np.uint32)[0], (what, t, hi, ost.scal)
-    gi, gv = state_view.window(sb, lay, m, kb)
+    gi, gv = state_view.canonical_rows(*state_view.window(sb, lay, m, kb))
     for s in range(max(1, t - m + 1), t + 1):
         r = s % m
         assert np.array_equal(gi[r], ost.G_idx[r]), f"window indices differ {what} t={t} row step {s}"
@@ -178,7 +179,9 @@ def test_fused_step(d, Bd, kb, m, steps, kind, wd):
 
 
 def test_fused_equals_two_kernels():
-    """The fused step and select + apply give the same bytes, step after step."""
+    """The fused step and select + apply give the same bytes, step after step
+    (the window rows as sets of pairs: the two paths list a row in different
+    orders)."""
     torch, MicroAdam, workloads = _mods()
     d, Bd, kb, m = 7 * 16384 + 4000, 16384, 164, 5
     w = workloads.Workload("pair", d, Bd, kb, m, "t3", 12, seed=4)
@@ -194,7 +197,10 @@ def test_fused_equals_two_kernels():
         mo.select(pb, g, sb, t=t, **hyper)
         mo.apply(pb, g, sb, t=t, **hyper)
         torch.cuda.synchronize()
-        assert torch.equal(sa[:20], sb[:20]) and torch.equal(sa[32:], sb[32:]), t
+        lay = mo.layout
+        assert torch.equal(sa[:20], sb[:20]), t
+        assert torch.equal(sa[lay.codes:lay.window], sb[lay.codes:lay.window]), t
+        assert state_view.same_window_sets(sa.cpu().numpy(), sb.cpu().numpy(), lay), t
         assert torch.equal(pa, pb), t
 
 

@@ -1,9 +1,10 @@
 """The sharded step on one GPU: shard handles of one vector, run one after the
 other with the 8-byte (-delta, Delta) exchange done as a device-side MAX (what
 the all-reduce of a multi-rank run computes), against the oracle run on the
-whole vector, every step: the shards' codes, window rows and scalars bit for
-bit, their parameters within 1e-5; and bit for bit against the unsharded
-step. No kernel waits on another; each launch completes on its own."""
+whole vector, every step: the shards' codes, window rows (as sets of pairs)
+and scalars bit for bit, their parameters within 1e-5; and bit for bit against
+the unsharded step (window rows as sets of pairs). No kernel waits on another;
+each launch completes on its own."""
 import numpy as np
 import pytest
 
@@ -62,9 +63,9 @@ def test_shards_reproduce_whole_vector(world):
         wv = win.view(np.uint32).reshape(lw.blocks, m, kp)[:, :, :kb].transpose(1, 0, 2)
         for s_ in range(max(1, t - m + 1), t + 1):
             r = s_ % m
-            assert np.array_equal((wv[r] & 0xFFFF).astype(np.uint16).view(np.int16),
-                                  ost.G_idx[r]), (t, s_)
-            assert np.array_equal((wv[r] >> 16).astype(np.uint16), ost.G_val[r]), (t, s_)
+            gi, gv = state_view.canonical_words(wv[r])
+            assert np.array_equal(gi, ost.G_idx[r]), (t, s_)
+            assert np.array_equal(gv, ost.G_val[r]), (t, s_)
         p = torch.cat(p_sh).cpu().numpy().astype(np.float64)
         tol = 1e-5 * np.maximum(np.abs(p_ref.astype(np.float64)), hyper["lr"])
         assert np.all(np.abs(p - p_ref) <= tol), t
@@ -73,7 +74,11 @@ def test_shards_reproduce_whole_vector(world):
                        for s, st in zip(shards, st_sh)])
     assert torch.equal(codes, st_whole[lw.codes: lw.codes + (d + 1) // 2])
     win = torch.cat([st[s.layout.window: s.layout.bytes] for s, st in zip(shards, st_sh)])
-    assert torch.equal(win, st_whole[lw.window: lw.bytes])
+    # the whole vector takes the fused step, which lists a row in another order
+    wi, wv = state_view.canonical_words(win.cpu().numpy().view(np.uint32).reshape(-1, lw.row_stride))
+    ri, rv = state_view.canonical_words(
+        st_whole[lw.window: lw.bytes].cpu().numpy().view(np.uint32).reshape(-1, lw.row_stride))
+    assert np.array_equal(wi, ri) and np.array_equal(wv, rv)
     for st in st_sh:
         assert torch.equal(st[:16], st_whole[:16])
     assert torch.equal(torch.cat(p_sh), p_whole)
