@@ -24,7 +24,7 @@ namespace {
 template <int T, bool VEC, bool FULL>
 __device__ __forceinline__ void codec_pass(const StepArgs& A, int64_t start, int base, int L,
                                            const uint32_t* sel, const char* lvb, float dn,
-                                           float inv16,
+                                           float inv16, uint32_t big0,
                                            const uint4 (&gv)[kChunks],
                                            const uint32_t (&cv)[kChunks]) {
   const int tid = threadIdx.x;
@@ -52,7 +52,7 @@ __device__ __forceinline__ void codec_pass(const StepArgs& A, int64_t start, int
             __float_as_uint(*reinterpret_cast<const float*>(lvb + 4 * (b & 15u)));
         a2[i] = f2_add_rn(g2, l2);
       }
-      pack = quantize8(a2, selbits, x, f2_pack(dn, dn), f2_pack(inv16, inv16));
+      pack = quantize8(a2, selbits, x, f2_pack(dn, dn), f2_pack(inv16, inv16), big0);
     } else {
       const int64_t gidx = G.base_index + start + eb;
       const uint64_t ga = (uint64_t)gidx >> 3;
@@ -140,17 +140,18 @@ __global__ void __launch_bounds__(T, (T == 256 ? MUA_APPLY_CTAS_256 : (T <= 512 
   const float inv16 =
       (Dn == dn) ? 0.0f : __fmul_rn(__fdiv_rn(15.0f, __fsub_rn(Dn, dn)), 65536.0f);
   const char* lvb = reinterpret_cast<const char*>(s_lv);
+  const uint32_t big0 = quantize_big_zero(dn, inv16);
   // The block in passes of kPass elements (the first pass's loads were issued
   // above).
   if (full) {
     for (int base = 0; base < L; base += kPass) {
       if (base > 0) load_block<T, VEC, true>(A.grads, A.codes, start + base, L - base, tid, gv, cv);
-      codec_pass<T, VEC, true>(A, start, base, L, sel, lvb, dn, inv16, gv, cv);
+      codec_pass<T, VEC, true>(A, start, base, L, sel, lvb, dn, inv16, big0, gv, cv);
     }
   } else {
     for (int base = 0; base < L; base += kPass) {
       if (base > 0) load_block<T, VEC>(A.grads, A.codes, start + base, L - base, tid, gv, cv);
-      codec_pass<T, VEC, false>(A, start, base, L, sel, lvb, dn, inv16, gv, cv);
+      codec_pass<T, VEC, false>(A, start, base, L, sel, lvb, dn, inv16, big0, gv, cv);
     }
   }
   __syncthreads();  // (6) AdamStats update of block j

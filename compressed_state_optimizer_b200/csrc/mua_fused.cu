@@ -265,6 +265,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
   const float inv16 =
       (Dn == dn) ? 0.0f : __fmul_rn(__fdiv_rn(15.0f, __fsub_rn(Dn, dn)), 65536.0f);
   const uint64_t dn2 = f2_pack(dn, dn), inv2 = f2_pack(inv16, inv16);
+  const uint32_t big0 = quantize_big_zero(dn, inv16);
 #pragma unroll
   for (int c = 0; c < kChunks; ++c) {
     const int e0 = elem_index<T>(c, tid, 0);
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         a2[i] = ((uint64_t)ab[c * kChunk + 2 * i + 1] << 32) | ab[c * kChunk + 2 * i];
-      pack = quantize8(a2, selbits, x, dn2, inv2);
+      pack = quantize8(a2, selbits, x, dn2, inv2, big0);
     } else {
       const int64_t gidx = G.base_index + start + e0;
 #pragma unroll

@@ -278,29 +278,36 @@ __device__ __forceinline__ uint32_t quantize_code_hi(float s16, uint32_t r) {
   return __viaddmin_u32(big, r, 0x4B0FFFFFu);  // min(big + r, code 15)
 }
 
+// The fixed-point value `big` (below) of a = +0, the value every selected
+// entry quantizes from: the same operations on the same operands.
+__device__ __forceinline__ uint32_t quantize_big_zero(float dn, float inv16) {
+  return __float_as_uint(__fadd_rz(__fmul_rn(__fsub_rn(0.0f, dn), inv16), 8388608.0f));
+}
+
 // Stage (4) for the 8 elements of a chunk [MicroAdam ¶1]: a2[i] holds the
 // pair (a of element 2i, a of element 2i + 1) as fp32 bits (low, high);
-// elements whose bit is set in `selbits` were selected and quantize as +0;
-// x is the chunk's Philox4x32-10 output (element e draws the (e mod 2)-th
-// 16-bit half of word e / 2); dn2 and inv2 hold (delta, delta) and
-// (2^16 * 15 / (Delta - delta)) twice. Returns the 8 codes packed into one
-// word, element e in bits 4e .. 4e + 3.
+// elements whose bit is set in `selbits` were selected and quantize as +0
+// (their `big` is big0 = quantize_big_zero(delta, inv16)); x is the chunk's
+// Philox4x32-10 output (element e draws the (e mod 2)-th 16-bit half of word
+// e / 2); dn2 and inv2 hold (delta, delta) and (2^16 * 15 / (Delta - delta))
+// twice. Returns the 8 codes packed into one word, element e in bits
+// 4e .. 4e + 3.
 //   s16 = (a - delta) * inv16, big = 2^23 + s16 rounded toward zero, so the low
 //   mantissa of big is floor(s16); the code is min(15, (floor(s16) + r) >> 16),
 //   which sits in bits 16..19 of min(big + r, 0x4B0FFFFF), i.e. in byte 2.
 __device__ __forceinline__ uint32_t quantize8(const uint64_t (&a2)[4], uint32_t selbits,
-                                              const uint4& x, uint64_t dn2, uint64_t inv2) {
+                                              const uint4& x, uint64_t dn2, uint64_t inv2,
+                                              uint32_t big0) {
   const uint64_t magic2 = f2_pack(8388608.0f, 8388608.0f);
   uint32_t hi[kChunk];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    uint64_t a = a2[i];
-    if ((selbits >> (2 * i)) & 1u) a &= 0xFFFFFFFF00000000ull;  // selected: a = +0
-    if ((selbits >> (2 * i + 1)) & 1u) a &= 0x00000000FFFFFFFFull;
-    const uint64_t big2 = f2_add_rz(f2_mul_rn(f2_sub_rn(a, dn2), inv2), magic2);
+    const uint64_t big2 = f2_add_rz(f2_mul_rn(f2_sub_rn(a2[i], dn2), inv2), magic2);
+    const uint32_t b0 = ((selbits >> (2 * i)) & 1u) ? big0 : (uint32_t)big2;
+    const uint32_t b1 = ((selbits >> (2 * i + 1)) & 1u) ? big0 : (uint32_t)(big2 >> 32);
     const uint32_t xw = chunk_word(x, i);
-    hi[2 * i] = __viaddmin_u32((uint32_t)big2, xw & 0xFFFFu, 0x4B0FFFFFu);
-    hi[2 * i + 1] = __viaddmin_u32((uint32_t)(big2 >> 32), xw >> 16, 0x4B0FFFFFu);
+    hi[2 * i] = __viaddmin_u32(b0, xw & 0xFFFFu, 0x4B0FFFFFu);
+    hi[2 * i + 1] = __viaddmin_u32(b1, xw >> 16, 0x4B0FFFFFu);
   }
   // Byte 2 of each (0..15, the code): even elements into one word, odd ones
   // into another, then one nibble interleave.

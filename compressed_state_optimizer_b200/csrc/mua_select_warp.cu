@@ -431,21 +431,26 @@ __device__ __forceinline__ void warp_radix(int hi, uint32_t prefix, int k, uint3
 // The threshold sample: 64 chunks of 8 elements spread over the block (chunk
 // c at element (c * (L / 64)) & ~7), each lane's two largest keys, sorted
 // descending across the warp by a bitonic network (element r of the order in
-// lane r / 2, slot r % 2). Returns the keys at rank `r` and at rank 63.
+// lane r / 2, slot r % 2). Returns the keys at rank `r` and at rank 63. The
+// loads (sample_load) go out before the level table is ready.
 template <bool VEC>
-__device__ __forceinline__ void sample_threshold(const StepArgs& A, int64_t start, int L,
-                                                 int r, int lane,
-                                                 uint32_t& tau_first, uint32_t& tau_retry) {
+__device__ __forceinline__ void sample_load(const StepArgs& A, int64_t start, int L, int lane,
+                                            uint4 (&gv)[2], uint32_t (&cv)[2]) {
+  const int cstride = (L / 64) & ~7;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+    load_step<VEC>(A.grads, A.codes, start, L, (lane + 32 * h) * cstride, gv[h], cv[h]);
+}
+__device__ __forceinline__ void sample_threshold(const uint4 (&gv)[2], const uint32_t (&cv)[2],
+                                                 int L, int r, int lane, uint32_t& tau_first,
+                                                 uint32_t& tau_retry) {
   const int cstride = (L / 64) & ~7;
   uint32_t t1 = 0u, t2 = 0u;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int e0 = (lane + 32 * h) * cstride;
-    uint4 gv;
-    uint32_t cv;
-    load_step<VEC>(A.grads, A.codes, start, L, e0, gv, cv);
     uint32_t ab[kChunk];
-    dequant8(gv, cv, e0, L, ab);
+    dequant8(gv[h], cv[h], e0, L, ab);
 #pragma unroll
     for (int e = 0; e < kChunk; ++e) {
       const uint32_t key = ab[e] & 0x7FFFFFFFu;
@@ -523,6 +528,26 @@ __global__ void __launch_bounds__(WARPS * 32, MINB)
   CtaSmem<CAP, WARPS>& S = *reinterpret_cast<CtaSmem<CAP, WARPS>*>(dyn);
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const Geometry& G = A.g;
+  const int j = blockIdx.x * WARPS + wid;
+  const bool live = j < G.nb;
+  int64_t start = 0;
+  int L = 0;
+  if (live) block_span(A, j, start, L);
+  const int k = live ? block_k(G, L) : 0;
+  const bool cand = live && L >= 1024 && L <= LMAX && 8 * k <= L;
+  // The block's L2 prefetch and the threshold sample's loads go out first:
+  // neither needs the level table.
+  uint4 sg[2];
+  uint32_t sc[2];
+  if (cand) {
+    if (VEC && (L & 255) == 0) {  // the streaming pass's data, on its way into L2
+      const int n = min(MUA_SELECT_PREFETCH_STEPS, L >> 8);
+      const bool pf = lane == 0 && aligned16(A.grads + start) && aligned16(A.codes + (start >> 1));
+      prefetch_l2_if(pf, A.grads + start, 512u * n);
+      prefetch_l2_if(pf, A.codes + (start >> 1), 128u * n);
+    }
+    sample_load<VEC>(A, start, L, lane, sg, sc);
+  }
   {
     const float delta = 0.0f - __uint_as_float(A.hdr[A.pair_cur]);
     const float Delta = __uint_as_float(A.hdr[A.pair_cur + 1]);
@@ -530,14 +555,9 @@ __global__ void __launch_bounds__(WARPS * 32, MINB)
     fill_levels(s_levels, delta, unit);
   }
   __syncthreads();  // the only CTA barrier: the level table
-  const int j = blockIdx.x * WARPS + wid;
-  if (j >= G.nb) return;
+  if (!live) return;
   WarpSmem<CAP>& W = S.w[wid];
   uint32_t* const status = &A.hdr[kHdrStatus];
-  int64_t start;
-  int L;
-  block_span(A, j, start, L);
-  const int k = block_k(G, L);
   uint32_t* row = A.window + ((int64_t)j * G.m + A.row) * G.kp;
   const int nsteps = (L + 255) >> 8;
 
@@ -545,17 +565,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB)
   bool done = false;
 
   // ---------------- candidate path
-  if (L >= 1024 && L <= LMAX && 8 * k <= L) {
+  if (cand) {
     // rank of tau_lo among the 64 sampled values: ~2.5 % of the block above it
     const int r = min(63, (int)((1280u * (uint32_t)k + (uint32_t)L - 1u) / (uint32_t)L) - 1);
-    if (VEC && (L & 255) == 0) {  // the streaming pass's data, on its way into L2
-      const int n = min(MUA_SELECT_PREFETCH_STEPS, L >> 8);
-      const bool pf = lane == 0 && aligned16(A.grads + start) && aligned16(A.codes + (start >> 1));
-      prefetch_l2_if(pf, A.grads + start, 512u * n);
-      prefetch_l2_if(pf, A.codes + (start >> 1), 128u * n);
-    }
     uint32_t tau_first, tau_retry;
-    sample_threshold<VEC>(A, start, L, r, lane, tau_first, tau_retry);
+    sample_threshold(sg, sc, L, r, lane, tau_first, tau_retry);
 
     // One streaming pass per attempt (a second, with a lower tau_lo, only when
     // the first finds fewer than k candidates). An all-zero sample goes
