@@ -203,10 +203,11 @@ struct Lane {
 };
 
 // Makes room in a lane's region for one more 8-element step: while it holds
-// more than CAP - 8 entries, every entry with the smallest key is dropped into
-// the residual's min/max (the others are compacted) and the lane's threshold
-// rises above that key, so every key the lane ever drops is below its final
-// threshold.
+// more than CAP - 8 entries, every entry with one of its two smallest keys is
+// dropped into the residual's min/max (the others are compacted) and the
+// lane's threshold rises above those keys, so every key the lane ever drops
+// is below its final threshold. (Dropping two key values at a time halves
+// the calls of a lane whose elements keep crossing its threshold.)
 template <int CAP>
 __device__ __noinline__ Lane<CAP> make_room(Lane<CAP> st, uint32_t* status) {
   while (st.full()) {
@@ -214,10 +215,16 @@ __device__ __noinline__ Lane<CAP> make_room(Lane<CAP> st, uint32_t* status) {
     uint32_t m0 = kFull;
     for (int i = 0; i < n; ++i)
       m0 = min(m0, lds_cand(st.base + 128u * i, st.ibase + 64u * i).x & 0x7FFFFFFFu);
+    uint32_t m1 = kFull;  // the second smallest key, if any
+    for (int i = 0; i < n; ++i) {
+      const uint32_t key = lds_cand(st.base + 128u * i, st.ibase + 64u * i).x & 0x7FFFFFFFu;
+      if (key > m0) m1 = min(m1, key);
+    }
+    if (m1 != kFull) m0 = m1;
     uint32_t kept = 0u;
     for (int i = 0; i < n; ++i) {
       const uint2 e = lds_cand(st.base + 128u * i, st.ibase + 64u * i);
-      if ((e.x & 0x7FFFFFFFu) == m0) {
+      if ((e.x & 0x7FFFFFFFu) <= m0) {
         st.rmin = fminf(st.rmin, __uint_as_float(e.x));
         st.rmax = fmaxf(st.rmax, __uint_as_float(e.x));
       } else {
