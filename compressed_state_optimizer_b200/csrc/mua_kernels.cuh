@@ -446,11 +446,11 @@ __device__ __forceinline__ void update_prefetch_rows(const StepArgs& A, int j, u
 // and, if wd != 0, p <- p*(1 - lr*wd) on every other parameter of the block:
 // each parameter is read and written once, and a bf16 parameter (BF16) is
 // rounded once. The rows are staged in shared memory and a
-// bitmask + popcount prefix gives each index its union rank. The sums run one
-// row at a time, oldest row first: the indices of one row are distinct, so no
-// two threads touch one accumulator within a row, and every accumulator sees
-// its terms in the same order on every run. Called by all T threads, after a
-// barrier.
+// bitmask + popcount prefix gives each index its union rank. Two warps run
+// the sums one row at a time, oldest row first: the indices of one row are
+// distinct, so no two threads touch one accumulator within a row, and every
+// accumulator sees its terms in the same order on every run. Called by all
+// T threads, after a barrier.
 template <int T, bool BF16>
 __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t start, int L,
                                              uint8_t* smem, const float* s_w1,
@@ -535,22 +535,33 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
     pv0[b] = (r < U) ? load_param_sparse<BF16>(A, start + pidx[b]) : 0.0f;
   }
 
-  // The sums, one row at a time from the oldest: z <- z + beta^age * V.
-  for (int age = A.rows - 1; age >= 0; --age) {
-    const float c1 = s_w1[age], c2 = s_w2[age];
-    const uint32_t* Wr = W + age * G.kp;
-    for (int p = tid; p < G.kp; p += T) {
-      const uint32_t v = Wr[p];
-      const uint32_t r = v & 0xFFFFu;
-      if (r == 0xFFFFu) continue;
-      const float V = __uint_as_float(v & 0xFFFF0000u);
-      float2 z = acc[r];
-      z.x = __fadd_rn(z.x, __fmul_rn(c1, V));
-      z.y = __fadd_rn(z.y, __fmul_rn(c2, __fmul_rn(V, V)));
-      acc[r] = z;
+  // The sums, one row at a time from the oldest: z <- z + beta^age * V. Two
+  // warps do them, with a 64-thread barrier between rows (ten CTA-wide
+  // barriers cost the other warps more than the rows' work: measured); the
+  // rest of the CTA waits once, after the last row.
+  constexpr int kSum = T < 64 ? T : 64;
+  if (tid < kSum) {
+    for (int age = A.rows - 1; age >= 0; --age) {
+      const float c1 = s_w1[age], c2 = s_w2[age];
+      const uint32_t* Wr = W + age * G.kp;
+      for (int p = tid; p < G.kp; p += kSum) {
+        const uint32_t v = Wr[p];
+        const uint32_t r = v & 0xFFFFu;
+        if (r == 0xFFFFu) continue;
+        const float V = __uint_as_float(v & 0xFFFF0000u);
+        float2 z = acc[r];
+        z.x = __fadd_rn(z.x, __fmul_rn(c1, V));
+        z.y = __fadd_rn(z.y, __fmul_rn(c2, __fmul_rn(V, V)));
+        acc[r] = z;
+      }
+      if constexpr (kSum == 32) {
+        __syncwarp();
+      } else {
+        asm volatile("bar.sync 1, %0;" ::"n"(kSum) : "memory");  // the summing warps only
+      }
     }
-    __syncthreads();
   }
+  __syncthreads();
 
   // Parameter update on the union: u = m_hat/(eps+sqrt(v_hat)) with the
   // hardware square root and reciprocal approximations (a few ulp, far inside
