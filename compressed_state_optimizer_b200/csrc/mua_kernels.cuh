@@ -535,33 +535,44 @@ __device__ __forceinline__ void block_update(const StepArgs& A, int j, int64_t s
     pv0[b] = (r < U) ? load_param_sparse<BF16>(A, start + pidx[b]) : 0.0f;
   }
 
-  // The sums, one row at a time from the oldest: z <- z + beta^age * V. Two
-  // warps do them, with a 64-thread barrier between rows (ten CTA-wide
-  // barriers cost the other warps more than the rows' work: measured); the
-  // rest of the CTA waits once, after the last row.
+  // The sums, one row at a time from the oldest: z <- z + beta^age * V.
+  auto sum_row = [&](int age, int first, int stride) {
+    const float c1 = s_w1[age], c2 = s_w2[age];
+    const uint32_t* Wr = W + age * G.kp;
+    for (int p = first; p < G.kp; p += stride) {
+      const uint32_t v = Wr[p];
+      const uint32_t r = v & 0xFFFFu;
+      if (r == 0xFFFFu) continue;
+      const float V = __uint_as_float(v & 0xFFFF0000u);
+      float2 z = acc[r];
+      z.x = __fadd_rn(z.x, __fmul_rn(c1, V));
+      z.y = __fadd_rn(z.y, __fmul_rn(c2, __fmul_rn(V, V)));
+      acc[r] = z;
+    }
+  };
+  // Up to 16 rows, two warps do them with a 64-thread barrier between rows
+  // (CTA-wide barriers cost the other warps more than the rows' work:
+  // measured), and the CTA meets once after the last row; longer windows
+  // spread each row over the whole CTA.
   constexpr int kSum = T < 64 ? T : 64;
-  if (tid < kSum) {
-    for (int age = A.rows - 1; age >= 0; --age) {
-      const float c1 = s_w1[age], c2 = s_w2[age];
-      const uint32_t* Wr = W + age * G.kp;
-      for (int p = tid; p < G.kp; p += kSum) {
-        const uint32_t v = Wr[p];
-        const uint32_t r = v & 0xFFFFu;
-        if (r == 0xFFFFu) continue;
-        const float V = __uint_as_float(v & 0xFFFF0000u);
-        float2 z = acc[r];
-        z.x = __fadd_rn(z.x, __fmul_rn(c1, V));
-        z.y = __fadd_rn(z.y, __fmul_rn(c2, __fmul_rn(V, V)));
-        acc[r] = z;
-      }
-      if constexpr (kSum == 32) {
-        __syncwarp();
-      } else {
-        asm volatile("bar.sync 1, %0;" ::"n"(kSum) : "memory");  // the summing warps only
+  if (G.m <= 16) {
+    if (tid < kSum) {
+      for (int age = A.rows - 1; age >= 0; --age) {
+        sum_row(age, tid, kSum);
+        if constexpr (kSum == 32) {
+          __syncwarp();
+        } else {
+          asm volatile("bar.sync 1, %0;" ::"n"(kSum) : "memory");  // the summing warps only
+        }
       }
     }
+    __syncthreads();
+  } else {
+    for (int age = A.rows - 1; age >= 0; --age) {
+      sum_row(age, tid, T);
+      __syncthreads();
+    }
   }
-  __syncthreads();
 
   // Parameter update on the union: u = m_hat/(eps+sqrt(v_hat)) with the
   // hardware square root and reciprocal approximations (a few ulp, far inside
