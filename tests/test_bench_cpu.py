@@ -1,6 +1,7 @@
-"""bench.py's reference arm (the CPU oracle timed on a bounded sample) runs
-without a GPU and prints one JSON line with the fields of the benchmark
-contract."""
+"""Host-side pieces of the measurement: bench.py's reference arm (the CPU
+oracle timed on a bounded sample) runs without a GPU and prints one JSON line
+with the fields of the benchmark contract; the committed traffic files match
+the kernel sources; the test helper that compares window rows as sets."""
 import json
 import os
 import subprocess
@@ -36,3 +37,33 @@ def test_workload_names():
     assert bench.get_workload("llama2_7b").segments() is None
     assert bench.get_workload("llama2_7b_bf16").params == "bf16"
     assert bench.get_workload("llama2_7b").params == "f32"
+
+
+def test_traffic_files_match_the_sources():
+    """The committed DRAM-traffic files were captured on the current kernel
+    sources (else the bench line reports traffic as null) and hold a per-launch
+    figure consistent with their per-parameter one."""
+    import bench
+    for kern in ("select", "apply"):
+        tr = bench.profiled_traffic(kern, "llama2_7b")
+        assert tr is not None, kern
+        path = os.path.join(ROOT, "profiles", f"traffic_{kern}_llama2_7b.txt")
+        kv = dict(line.split(":", 1) for line in open(path) if ":" in line)
+        per = float(kv["dram_bytes_per_param"])
+        assert abs(tr - per * 6738415616) / tr < 1e-3
+        assert 2.5 <= per < 12.0  # at least the gradient and code bytes
+
+
+def test_canonical_rows_orders_pairs_by_index():
+    """Window rows compared as sets: pairs sorted by index, empty slots last,
+    values moved with their indices."""
+    import numpy as np
+    import state_view
+    idx = np.array([[5, 1, -1, 3], [-1, 7, -1, 2]], dtype=np.int16)
+    val = np.array([[50, 10, 0, 30], [0, 70, 0, 20]], dtype=np.uint16)
+    gi, gv = state_view.canonical_rows(idx, val)
+    assert gi.tolist() == [[1, 3, 5, -1], [2, 7, -1, -1]]
+    assert gv.tolist() == [[10, 30, 50, 0], [20, 70, 0, 0]]
+    words = idx.view(np.uint16).astype(np.uint32) | (val.astype(np.uint32) << 16)
+    wi, wv = state_view.canonical_words(words)
+    assert np.array_equal(wi, gi) and np.array_equal(wv, gv)
