@@ -505,23 +505,42 @@ def run_e2e(args, step, mo, state, grads, t, w, dev, world, local_rank):
                 "h2d_bytes_per_step": need, "d2h_bytes_per_step": 12}
     host = torch.empty(grads[0].numel(), dtype=torch.bfloat16, pin_memory=True)
     host.copy_(grads[0])
-    dev_g = torch.empty_like(grads[0])
+    # Two device buffers: step i's gradients cross the host link on a copy
+    # stream while step i - 1 computes (every copy inside the timed region).
+    bufs = [torch.empty_like(grads[0]), torch.empty_like(grads[0])]
     back = torch.empty(12, dtype=torch.uint8, pin_memory=True)
     stream = torch.cuda.current_stream(dev)
+    copy_stream = torch.cuda.Stream(dev)
     steps = max(3, min(args.steps, 10))
     for _ in range(2):
         t += 1
-        dev_g.copy_(host, non_blocking=True)
-        step(t, dev_g)
+        bufs[0].copy_(host, non_blocking=True)
+        step(t, bufs[0])
     if world > 1:
         dist.barrier(device_ids=[local_rank])
     torch.cuda.synchronize(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    copied = [torch.cuda.Event(), torch.cuda.Event()]
+    used = [torch.cuda.Event(), torch.cuda.Event()]
+
+    def issue_copy(i):
+        k = i % 2
+        if i >= 2:
+            copy_stream.wait_event(used[k])  # step i - 2 is done with this buffer
+        with torch.cuda.stream(copy_stream):
+            bufs[k].copy_(host, non_blocking=True)
+        copied[k].record(copy_stream)
+
     a.record(stream)
-    for _ in range(steps):
+    copy_stream.wait_event(a)
+    issue_copy(0)
+    for i in range(steps):
+        if i + 1 < steps:
+            issue_copy(i + 1)
         t += 1
-        dev_g.copy_(host, non_blocking=True)
-        step(t, dev_g)
+        stream.wait_event(copied[i % 2])
+        step(t, bufs[i % 2])
+        used[i % 2].record(stream)
         back.copy_(state[:12], non_blocking=True)
     b.record(stream)
     torch.cuda.synchronize(dev)
