@@ -128,7 +128,10 @@ int64_t mua_state_bytes(mua_t h);
  * mua_state_layout — write the MUA_LAYOUT_FIELDS int64 values above into the
  * host array out. The window is uint32[n_b][m][row_stride]: entry = int16 I
  * (low half; 0xFFFF = empty slot) | bf16 V << 16; row (t mod m) of block j
- * holds the block's Top-k of step t in ascending index order. The header
+ * holds the block's Top-k of step t: its k entries first, in an order the
+ * kernels fix from the data alone (the same bytes on every run; the method
+ * does not order a row, and no later use of it depends on the order), then
+ * empty slots. The header
  * holds two (-delta, Delta) fp32 pairs at words 0-1 and 2-3 (pair t mod 2 is
  * step t's (delta_t, Delta_t)), the status word at word 4 and the fused step's
  * barrier count at word 5 (reset by every fused step).
